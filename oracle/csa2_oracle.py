@@ -1,0 +1,413 @@
+"""CSA2 oracle: a plain, slow, float64 CPU statement of what the CSA2 hot path computes.
+
+TEST INFRASTRUCTURE ONLY.  Nothing in the product imports this module: only
+``tests/``, ``__graft_entry__.smoke()`` and ``bench.py`` (its ``cpu_baseline``
+leg and ``--impl reference`` arm) may call it.  It shares no code, table or
+constant with the CUDA library, and it never reads anything the CUDA path
+wrote: every function takes plain numpy arrays of input *values* and returns
+float64 results.
+
+Sources (the pages carry the prose; every formula on them was lost in text
+extraction, so where a step is left open the plainest reading is taken and
+named in the function's docstring):
+
+* "读完这篇，你就搞懂 DeepSeek v4 了" (note.crab.center, DeepSeek V4 explainer),
+  sections 闪电索引机制 (lightning indexer, eq. 8), 注意力计算 (shared-KV
+  attention, eq. 9), HCA 压缩机制 (eq. 10) and 权重矩阵S (eq. 11), the
+  "会议记录员 ... 前后两场小会" metaphor for CSA compression, and
+  FP4量化感知训练 (FP4 for indexer q/K, BF16 scores).
+* DeepSeek V4.1 Flash video transcript (prism.simon-ai.net, article 7827),
+  the CSA2 paragraph (Full / Reindex / Reuse) and the hierarchical sparse
+  indexer paragraph (candidate pool of about 16,384 positions).
+* "Recall之王 祭出Reuse" (10100.com), the CSA2 bullet list: Hierarchical
+  Sparse Indexer and FP4 主KV缓存 (E2M1 values, one E4M3 scale per 16
+  channels).
+
+Pinning status (what checks this file against something other than itself is
+listed in tests/test_oracle_pins.py):
+  bf16 rounding, compression, index score, top-k / pool, attention, FP4
+  pack/unpack, and the three layer modes are all pinned.  The pages' model-level
+  figures (about 890 bytes per token, 437x smaller than V1) are "parity
+  unpinned": they cannot be derived from the pages.
+"""
+from __future__ import annotations
+
+import numpy as np
+
+# ----------------------------------------------------------------------------
+# bfloat16 values
+# ----------------------------------------------------------------------------
+
+
+def bf16_bits_to_float(bits: np.ndarray) -> np.ndarray:
+    """Decode raw bfloat16 bit patterns (uint16) to float64 values (exact)."""
+    bits = np.asarray(bits, dtype=np.uint16)
+    return (bits.astype(np.uint32) << np.uint32(16)).view(np.float32).astype(np.float64)
+
+
+_BF16_MAX = float(np.ldexp(255.0, 120))  # largest finite bfloat16, (2 - 2**-7) * 2**127
+
+
+def round_to_bf16(x: np.ndarray) -> np.ndarray:
+    """Round float64 values to the nearest bfloat16 value, ties to even.
+
+    bfloat16 keeps 8 significant bits, its smallest normal is 2**-126 and its
+    subnormal quantum is 2**-133.  The result is returned as float64 values.
+    Rounding is done once, directly from float64 (no float32 detour, so there
+    is no double rounding).
+    """
+    x = np.asarray(x, dtype=np.float64)
+    out = np.array(x, dtype=np.float64, copy=True)
+    fin = np.isfinite(x)
+    xf = x[fin]
+    _, e = np.frexp(xf)                  # xf = mant * 2**e with 0.5 <= |mant| < 1
+    q = np.maximum(e - 8, -133)          # exponent of one unit in the last place
+    r = np.ldexp(np.round(np.ldexp(xf, -q)), q)   # np.round: half to even
+    # overflow: anything that rounds past the largest finite value becomes inf
+    over = np.abs(r) > _BF16_MAX
+    r[over] = np.copysign(np.inf, xf[over])
+    out[fin] = r
+    return out
+
+
+# ----------------------------------------------------------------------------
+# (a1) token -> entry compression
+# ----------------------------------------------------------------------------
+
+
+def compress(c: np.ndarray, z: np.ndarray, bias: np.ndarray, m: int,
+             has_left_halo: bool = False):
+    """CSA token-dimension compression.
+
+    V4 explainer: CSA's "meeting recorder" writes each summary while attending
+    to *two consecutive* small meetings (the HCA paragraph says HCA differs
+    exactly by *not* joining two consecutive groups); eq. (11) defines the
+    weight matrix S as a softmax of the projected logits Z plus a learned
+    bias matrix B, and the entry is the S-weighted sum of the value
+    projections C.  Readings taken where the formula is lost:
+
+    * entry j (0-based) covers blocks j-1 and j, i.e. tokens
+      [(j-1)m, (j+1)m); tokens before the first one are absent (their weight
+      is zero) unless ``has_left_halo``, in which case the first m rows of
+      ``c``/``z`` are the block just before the chunk;
+    * the softmax runs per channel over the window's token positions;
+    * ``bias[w, ch]`` is indexed by the position w in 0..2m-1 inside the
+      window (w < m: earlier block);
+    * each token has one (c_t, z_t); only the bias depends on the window.
+
+    Args (values as float64):
+      c: [B, T_in, D] value projections (bf16 values)
+      z: [B, T_in, D] logits (fp32 values)
+      bias: [2m, D]
+    Returns (e_exact, e_bf16), both float64 [B, N, D] with N = (T_in - halo)//m;
+    a trailing partial block forms no entry.
+    """
+    c = np.asarray(c, dtype=np.float64)
+    z = np.asarray(z, dtype=np.float64)
+    bias = np.asarray(bias, dtype=np.float64)
+    assert bias.shape[0] == 2 * m
+    halo = m if has_left_halo else 0
+    B, T_in, D = c.shape
+    N = (T_in - halo) // m
+    e = np.zeros((B, N, D), dtype=np.float64)
+    for j in range(N):
+        first = (j - 1) * m + halo          # array row of window position 0
+        w0 = 0 if first >= 0 else m         # window positions that exist
+        rows = slice(first + w0, first + 2 * m)
+        logits = z[:, rows, :] + bias[w0:2 * m][None, :, :]
+        top = logits.max(axis=1, keepdims=True)
+        p = np.exp(logits - top)
+        p /= p.sum(axis=1, keepdims=True)
+        e[:, j, :] = (p * c[:, rows, :]).sum(axis=1)
+    return e, round_to_bf16(e)
+
+
+# ----------------------------------------------------------------------------
+# (a2) lightning-indexer score
+# ----------------------------------------------------------------------------
+
+
+def index_scores(q: np.ndarray, w: np.ndarray, k: np.ndarray,
+                 n_visible: np.ndarray | None = None,
+                 pool: np.ndarray | None = None,
+                 act: str = "relu") -> np.ndarray:
+    """Lightning-indexer relevance score (V4 explainer, 闪电索引机制, eq. 8).
+
+    The page says the indexer works like DeepSeek V3.2's DSA: every query
+    token gets a score against every compressed entry, each indexer head's
+    score is weighted by a per-head weight w (projected from the query's
+    hidden state) and the weighted head scores are summed.  Reading: the DSA
+    form  s[j] = sum_h w[h] * act(q[h] . k[j])  with act = ReLU ("identity"
+    is also offered).
+
+    Args:
+      q: [B, Q, H, d], w: [B, Q, H], k: [B, N, d]   (float64 values)
+      n_visible: [B, Q] or None.  Entries j >= n_visible[b, q] are not
+        scored (Full layer, causal prefill).  None = all N visible.
+      pool: [B, Q, P] entry indices (-1 = empty slot) or None.  With a pool
+        the score of pool slot p is the score of entry pool[b, q, p]
+        (hierarchical indexer: a Reindex layer scores only inside the pool the
+        Full layer built).
+    Returns float64 [B, Q, N] (no pool) or [B, Q, P]; unscored slots are -inf.
+    """
+    q = np.asarray(q, dtype=np.float64)
+    w = np.asarray(w, dtype=np.float64)
+    k = np.asarray(k, dtype=np.float64)
+    B, Q, H, d = q.shape
+    N = k.shape[1]
+    L = N if pool is None else pool.shape[2]
+    out = np.full((B, Q, L), -np.inf, dtype=np.float64)
+    for b in range(B):
+        for t in range(Q):
+            if pool is None:
+                ids = np.arange(N)
+                nv = N if n_visible is None else int(n_visible[b, t])
+                valid = ids < nv
+            else:
+                ids = np.asarray(pool[b, t], dtype=np.int64)
+                valid = ids >= 0
+            rows = k[b][np.where(valid, ids, 0)]          # [L, d]
+            head_dots = rows @ q[b, t].T                  # [L, H]: q_h . k_j
+            if act == "relu":
+                head_dots = np.maximum(head_dots, 0.0)
+            elif act != "identity":
+                raise ValueError(act)
+            s = head_dots @ w[b, t]                       # sum_h w_h * act(.)
+            out[b, t] = np.where(valid, s, -np.inf)
+    return out
+
+
+# ----------------------------------------------------------------------------
+# (a3) top-k selection (and the hierarchical pool)
+# ----------------------------------------------------------------------------
+
+
+def select_top(scores: np.ndarray, count: int,
+               tie_key: np.ndarray | None = None) -> np.ndarray:
+    """Positions of the ``count`` best scores of each row.
+
+    V4 explainer (闪电索引机制): keep the k most relevant entries.  Readings:
+    the order is score descending, ties broken by the smaller tie key (the
+    entry index; by default the position itself); -inf slots are never
+    chosen; the result lists the chosen positions in ascending order and is
+    padded with -1 when fewer than ``count`` are selectable.
+
+    scores: [..., L]; tie_key: same shape or None.  Returns int64 [..., count].
+    """
+    scores = np.asarray(scores, dtype=np.float64)
+    lead = scores.shape[:-1]
+    L = scores.shape[-1]
+    flat = scores.reshape(-1, L)
+    keys = (np.broadcast_to(np.arange(L), flat.shape) if tie_key is None
+            else np.asarray(tie_key).reshape(-1, L))
+    res = np.full((flat.shape[0], count), -1, dtype=np.int64)
+    for r in range(flat.shape[0]):
+        s = flat[r]
+        ok = np.where(s > -np.inf)[0]
+        order = np.lexsort((keys[r][ok], -s[ok]))   # primary: -score, then key
+        chosen = np.sort(ok[order[:count]])
+        res[r, :chosen.size] = chosen
+    return res.reshape(*lead, count)
+
+
+def gather_pool_ids(pool: np.ndarray, pos: np.ndarray) -> np.ndarray:
+    """Map positions inside a pool back to entry indices (-1 stays -1)."""
+    out = np.full(pos.shape, -1, dtype=np.int64)
+    B, Q, _ = pos.shape
+    for b in range(B):
+        for t in range(Q):
+            p = pos[b, t]
+            ok = p >= 0
+            out[b, t, ok] = pool[b, t, p[ok]]
+    return out
+
+
+# ----------------------------------------------------------------------------
+# (a4) shared-KV sparse attention
+# ----------------------------------------------------------------------------
+
+
+def sparse_attn(q: np.ndarray, kv: np.ndarray, topk: np.ndarray, scale: float):
+    """Shared-KV attention over the selected entries (V4 explainer, 注意力计算,
+    eq. 9): ordinary softmax attention in which every query head uses the
+    same compressed entries C as keys and as values, restricted to the top-k
+    entries the indexer chose.
+
+    out[h] = sum_{j in S} softmax_j(scale * q[h] . kv[j]) * kv[j]
+    lse[h] = log sum_{j in S} exp(scale * q[h] . kv[j])
+
+    Args: q [B, Q, Ha, D], kv [B, N, D] (values), topk [B, Q, k] entry ids
+    (-1 = empty).  An empty selection gives out = 0 and lse = -inf.
+    Returns (o_exact [B,Q,Ha,D], o_bf16, lse [B,Q,Ha]) as float64.
+    """
+    q = np.asarray(q, dtype=np.float64)
+    kv = np.asarray(kv, dtype=np.float64)
+    B, Q, Ha, D = q.shape
+    o = np.zeros((B, Q, Ha, D), dtype=np.float64)
+    lse = np.full((B, Q, Ha), -np.inf, dtype=np.float64)
+    for b in range(B):
+        for t in range(Q):
+            ids = np.asarray(topk[b, t], dtype=np.int64)
+            ids = ids[ids >= 0]
+            if ids.size == 0:
+                continue
+            ent = kv[b][ids]                          # [k', D]
+            logits = scale * (q[b, t] @ ent.T)        # [Ha, k']
+            top = logits.max(axis=1, keepdims=True)
+            p = np.exp(logits - top)
+            l = p.sum(axis=1, keepdims=True)
+            o[b, t] = (p @ ent) / l
+            lse[b, t] = (top + np.log(l))[:, 0]
+    return o, round_to_bf16(o), lse
+
+
+# ----------------------------------------------------------------------------
+# (a5) FP4 main-KV format: E2M1 values, one E4M3 scale per 16 channels
+# ----------------------------------------------------------------------------
+
+FP4_BLOCK = 16
+
+
+def e2m1_value(code: np.ndarray) -> np.ndarray:
+    """E2M1 (1 sign, 2 exponent, 1 mantissa bit, exponent bias 1, no inf/NaN).
+
+    Exponent field 0 is subnormal (0 or 0.5); otherwise (1 + m/2) * 2**(e-1).
+    """
+    code = np.asarray(code, dtype=np.int64)
+    e = (code >> 1) & 3
+    mt = code & 1
+    mag = np.where(e == 0, 0.5 * mt, (1.0 + 0.5 * mt) * np.ldexp(1.0, e - 1))
+    return np.where(code & 8, -mag, mag)
+
+
+def e4m3_value(code: np.ndarray) -> np.ndarray:
+    """E4M3 (the 'fn' variant: bias 7, no inf, S.1111.111 is NaN, max 448)."""
+    code = np.asarray(code, dtype=np.int64)
+    e = (code >> 3) & 15
+    mt = code & 7
+    mag = np.where(e == 0, (mt / 8.0) * 2.0 ** -6,
+                   (1.0 + mt / 8.0) * np.ldexp(1.0, e - 7))
+    mag = np.where((e == 15) & (mt == 7), np.nan, mag)
+    return np.where(code & 128, -mag, mag)
+
+
+_E2M1_MAGS = e2m1_value(np.arange(8))          # codes 0..7: 0 .5 1 1.5 2 3 4 6
+_E4M3_POS = e4m3_value(np.arange(127))         # finite non-negative codes 0..126
+
+
+def _nearest_code(target: np.ndarray, grid: np.ndarray) -> np.ndarray:
+    """Index of the grid value nearest to each target; a tie between two
+    neighbours goes to the even index (ties-to-even on the code's last bit).
+    Distances are exact in float64 for the operands used here."""
+    dist = np.abs(target[..., None] - grid)
+    best = dist.min(axis=-1, keepdims=True)
+    tied = dist == best
+    even = (np.arange(grid.shape[-1]) % 2) == 0
+    pick_even = tied & even
+    has_even = pick_even.any(axis=-1)
+    return np.where(has_even, pick_even.argmax(axis=-1), tied.argmax(axis=-1))
+
+
+def fp4_pack(x: np.ndarray):
+    """Quantise rows to E2M1 codes with one E4M3 scale per 16 channels.
+
+    "Recall之王" CSA2 bullets: the FP4 main KV is E2M1 with one E4M3 scaling
+    factor per 16 channels.  Readings (the page fixes only the format):
+
+    * the block scale s is the E4M3 value nearest absmax/6 (6 = largest E2M1
+      magnitude), ties to even, saturating at 448.  It is found without a
+      division: s minimises |absmax - 6*s| over the finite E4M3 values;
+    * each code is the E2M1 value v minimising |x - v*s|, ties to the even
+      code, saturating at +-6; the sign bit copies x's sign (so -0.0 and
+      small negatives give 0x8);
+    * absmax = 0 gives scale code 0x00 and all-zero magnitudes;
+    * byte i of a row holds channel 2i in its low nibble, 2i+1 in its high
+      nibble; there is no second-level (per-tensor) scale.
+
+    x: [R, D] float64 values (bf16 values), D % 16 == 0.
+    Returns (codes uint8 [R, D/2], scales uint8 [R, D/16]).
+    """
+    x = np.asarray(x, dtype=np.float64)
+    R, D = x.shape
+    assert D % FP4_BLOCK == 0
+    blk = x.reshape(R, D // FP4_BLOCK, FP4_BLOCK)
+    amax = np.abs(blk).max(axis=-1)                      # [R, D/16]
+    scode = _nearest_code(amax, 6.0 * _E4M3_POS)         # 0..126
+    s = _E4M3_POS[scode]
+    mag_code = _nearest_code(np.abs(blk), _E2M1_MAGS[None, None, :] * s[..., None, None])
+    mag_code = np.where(s[..., None] == 0.0, 0, mag_code)
+    sign = np.signbit(blk).astype(np.int64) << 3
+    code = (mag_code | sign).reshape(R, D)
+    packed = (code[:, 0::2] | (code[:, 1::2] << 4)).astype(np.uint8)
+    return packed, scode.astype(np.uint8)
+
+
+def fp4_unpack(codes: np.ndarray, scales: np.ndarray) -> np.ndarray:
+    """Inverse of the format: x = e2m1(code) * e4m3(scale) (exact in bf16)."""
+    codes = np.asarray(codes, dtype=np.uint8)
+    R, half = codes.shape
+    lo = codes & 0x0F
+    hi = codes >> 4
+    code = np.empty((R, half * 2), dtype=np.int64)
+    code[:, 0::2] = lo
+    code[:, 1::2] = hi
+    s = e4m3_value(np.asarray(scales, dtype=np.int64))      # [R, D/16]
+    return e2m1_value(code) * np.repeat(s, FP4_BLOCK, axis=1)
+
+
+# ----------------------------------------------------------------------------
+# (a6) the three per-layer modes
+# ----------------------------------------------------------------------------
+
+
+def run_group(modes, layers, kv, index_k, k_top: int, scale: float,
+              pool_size: int = 0, n_visible=None, act: str = "relu"):
+    """Run one CSA2 layer group (video transcript, CSA2 paragraph; "Recall之王"
+    CSA2 bullets and Hierarchical Sparse Indexer).
+
+    * full:    score every visible entry with the layer's own indexer queries,
+               keep its own top-k (and, with pool_size > 0, the pool of the
+               pool_size best entries), attend.
+    * reindex: reuse the main KV and indexer K; score with the layer's own
+               queries, inside the pool when there is one, else over every
+               visible entry; keep a fresh top-k; attend.
+    * reuse:   run no indexer; attend with the most recent selection.
+
+    kv: [B, N, D] main-KV values (already dequantised when stored as FP4);
+    index_k: [B, N, d].  layers[i] holds 'q_attn' and, for full/reindex,
+    'q_index' and 'w_index'.  Returns a list of per-layer dicts with
+    'topk', 'pool' (full only), 'o' (exact), 'o_bf16', 'lse'.
+    """
+    results = []
+    topk = None
+    pool = None
+    for i, mode in enumerate(modes):
+        L = layers[i]
+        res = {"mode": mode}
+        if mode == "full":
+            s = index_scores(L["q_index"], L["w_index"], index_k,
+                             n_visible=n_visible, act=act)
+            topk = select_top(s, k_top)
+            pool = select_top(s, pool_size) if pool_size > 0 else None
+            res["pool"] = pool
+        elif mode == "reindex":
+            if topk is None:
+                raise ValueError("reindex before any full layer")
+            if pool is not None:
+                s = index_scores(L["q_index"], L["w_index"], index_k,
+                                 pool=pool, act=act)
+                pos = select_top(s, k_top, tie_key=np.where(pool >= 0, pool, 0))
+                topk = gather_pool_ids(pool, pos)
+            else:
+                s = index_scores(L["q_index"], L["w_index"], index_k,
+                                 n_visible=n_visible, act=act)
+                topk = select_top(s, k_top)
+        elif mode == "reuse":
+            if topk is None:
+                raise ValueError("reuse before any full layer")
+        else:
+            raise ValueError(mode)
+        o, o16, lse = sparse_attn(L["q_attn"], kv, topk, scale)
+        res.update(topk=topk, o=o, o_bf16=o16, lse=lse)
+        results.append(res)
+    return results
