@@ -1,0 +1,223 @@
+// Shared-KV sparse attention over the selected entries.
+// Source: "读完这篇，你就搞懂 DeepSeek v4 了", 注意力计算 (eq. 9): standard
+// attention in which every query head uses the same compressed entries as
+// keys and values, restricted to the indexer's top-k; FP4 rows ("Recall之王",
+// FP4 主KV缓存) are dequantised in the kernel.
+//
+// This file holds the CUDA-core kernel: one CTA per query, the query's heads
+// in shared memory, the selected rows staged 16 at a time (f32, padded
+// stride), an online softmax per head and the per-head outputs in registers.
+// It serves every shape; the tensor-core kernel in attn_tc.cu takes the
+// shapes it supports.  The reduction order per query is fixed (rows in list
+// order, 16 at a time), so a query's result does not depend on B or Q.
+#include "common.cuh"
+#include "launchers.h"
+
+namespace csa2 {
+
+csa2_status launch_sparse_attn_tc(const void* q, const csa2_kv& kv, const int32_t* topk, int B,
+                                  int Q, int Ha, int k, float scale, void* out, float* lse,
+                                  void* ws, size_t ws_bytes, cudaStream_t stream);
+size_t sparse_attn_tc_workspace(int B, int Q, int Ha, int D, int k, csa2_kv_fmt fmt);
+
+namespace {
+
+constexpr int kT = 256;
+constexpr int kR = 16;  // rows staged per step
+
+template <int HA, int DD>
+struct AttnSmem {
+  static constexpr int RS = DD + 1;  // padded f32 row stride: conflict-free column reads
+  static constexpr size_t q_words = HA * DD / 2;
+  static constexpr size_t bytes = q_words * 4 + size_t(kR) * RS * 4 + size_t(HA) * (kR + 1) * 4 +
+                                  3 * HA * 4 + kR * 4;
+};
+
+template <int HA, int DD, bool FP4>
+__global__ void __launch_bounds__(kT) attn_simt_kernel(
+    const uint16_t* __restrict__ q, const void* __restrict__ kv_data,
+    const uint8_t* __restrict__ kv_scales, int64_t n, const int32_t* __restrict__ topk, int k,
+    float scale, uint16_t* __restrict__ out, float* __restrict__ lse, int* err) {
+  using S = AttnSmem<HA, DD>;
+  constexpr int TPH = kT / HA;      // threads per head in the accumulation
+  constexpr int OPT = DD / TPH;     // outputs per thread
+  constexpr int PAIRS = HA * kR / kT;
+  static_assert(kT % HA == 0 && DD % TPH == 0 && (HA * kR) % kT == 0, "shape");
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  uint32_t* q_s = reinterpret_cast<uint32_t*>(smem_raw);
+  float* rows_s = reinterpret_cast<float*>(q_s + S::q_words);
+  float* p_s = rows_s + kR * S::RS;           // [HA][kR+1]
+  float* m_s = p_s + HA * (kR + 1);
+  float* l_s = m_s + HA;
+  float* a_s = l_s + HA;
+  int* id_s = reinterpret_cast<int*>(a_s + HA);
+
+  const int tid = threadIdx.x;
+  const int64_t seq = blockIdx.y;                                   // sequence b
+  const int64_t qi = seq * gridDim.x + blockIdx.x;                  // flat (b, q)
+  const uint32_t* qg = reinterpret_cast<const uint32_t*>(q + qi * HA * DD);
+  for (int i = tid; i < HA * DD / 2; i += kT) q_s[i] = qg[i];
+  for (int h = tid; h < HA; h += kT) { m_s[h] = -INFINITY; l_s[h] = 0.0f; }
+  const int h_o = tid / TPH, d_o = tid % TPH;
+  float acc[OPT];
+#pragma unroll
+  for (int i = 0; i < OPT; ++i) acc[i] = 0.0f;
+  const int32_t* ids = topk + qi * k;
+
+  for (int c0 = 0; c0 < k; c0 += kR) {
+    __syncthreads();   // previous step done with rows_s / p_s / id_s
+    if (tid < kR) {
+      int id = (c0 + tid < k) ? ids[c0 + tid] : -1;
+      if (id >= n || id < -1) { raise_dev_error(err, DEVERR_BOUNDS); id = -1; }
+      id_s[tid] = id;
+    }
+    __syncthreads();
+    // stage rows as f32 (zeros for empty slots)
+    if (!FP4) {
+      constexpr int V = DD / 8;   // uint4 per row
+      for (int i = tid; i < kR * V; i += kT) {
+        const int r = i / V, c = i % V;
+        const int id = id_s[r];
+        uint4 v = make_uint4(0, 0, 0, 0);
+        if (id >= 0)
+          v = __ldg(reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(kv_data) +
+                                                   (seq * n + id) * DD) + c);
+        float* dst = rows_s + r * S::RS + c * 8;
+        dst[0] = bf16_lo(v.x); dst[1] = bf16_hi(v.x); dst[2] = bf16_lo(v.y); dst[3] = bf16_hi(v.y);
+        dst[4] = bf16_lo(v.z); dst[5] = bf16_hi(v.z); dst[6] = bf16_lo(v.w); dst[7] = bf16_hi(v.w);
+      }
+    } else {
+      constexpr int NB = DD / 16;  // 16-channel blocks per row
+      for (int i = tid; i < kR * NB; i += kT) {
+        const int r = i / NB, blk = i % NB;
+        const int id = id_s[r];
+        float* dst = rows_s + r * S::RS + blk * 16;
+        if (id < 0) {
+#pragma unroll
+          for (int u = 0; u < 16; ++u) dst[u] = 0.0f;
+          continue;
+        }
+        const int64_t row = seq * n + id;
+        const uint2 cw = __ldg(reinterpret_cast<const uint2*>(
+                                   static_cast<const uint8_t*>(kv_data) + row * (DD / 2)) + blk);
+        const uint32_t sc = __ldg(kv_scales + row * NB + blk);
+        const uint32_t se = (sc >> 3) & 15u, sm = sc & 7u;
+        float s = (se == 0) ? static_cast<float>(sm) * 0x1p-9f
+                            : __uint_as_float(((se + 120u) << 23) | (sm << 20));
+        if (sc & 128u) s = -s;
+#pragma unroll
+        for (int u = 0; u < 16; ++u) {
+          const uint32_t c = ((u < 8 ? cw.x : cw.y) >> (4 * (u & 7))) & 15u;
+          const uint32_t e = (c >> 1) & 3u, mt = c & 1u;
+          float mag = (e == 0) ? 0.5f * mt : (1.0f + 0.5f * mt) * static_cast<float>(1u << (e - 1));
+          dst[u] = ((c & 8u) ? -mag : mag) * s;
+        }
+      }
+    }
+    __syncthreads();
+    // logits for (head, row) pairs
+#pragma unroll
+    for (int pi = 0; pi < PAIRS; ++pi) {
+      const int r = tid % kR;
+      const int h = tid / kR + (kT / kR) * pi;
+      float dot = 0.0f;
+      const float* row = rows_s + r * S::RS;
+      const uint32_t* qh = q_s + h * (DD / 2);
+#pragma unroll 8
+      for (int i = 0; i < DD / 2; ++i) {
+        const uint32_t qq = qh[i];
+        dot = fmaf(bf16_lo(qq), row[2 * i], dot);
+        dot = fmaf(bf16_hi(qq), row[2 * i + 1], dot);
+      }
+      p_s[h * (kR + 1) + r] = (id_s[r] >= 0) ? scale * dot : -INFINITY;
+    }
+    __syncthreads();
+    // online softmax update, one thread per head
+    for (int h = tid; h < HA; h += kT) {
+      float* ph = p_s + h * (kR + 1);
+      float mx = m_s[h];
+#pragma unroll
+      for (int r = 0; r < kR; ++r) mx = fmaxf(mx, ph[r]);
+      float alpha = 1.0f, l = l_s[h];
+      if (mx != -INFINITY) {
+        alpha = (m_s[h] == -INFINITY) ? 0.0f : expf(m_s[h] - mx);
+        l *= alpha;
+#pragma unroll
+        for (int r = 0; r < kR; ++r) {
+          const float p = (ph[r] == -INFINITY) ? 0.0f : expf(ph[r] - mx);
+          ph[r] = p;
+          l += p;
+        }
+      } else {
+#pragma unroll
+        for (int r = 0; r < kR; ++r) ph[r] = 0.0f;
+      }
+      m_s[h] = mx;
+      l_s[h] = l;
+      a_s[h] = alpha;
+    }
+    __syncthreads();
+    const float alpha = a_s[h_o];
+    const float* ph = p_s + h_o * (kR + 1);
+#pragma unroll
+    for (int i = 0; i < OPT; ++i) acc[i] *= alpha;
+#pragma unroll
+    for (int r = 0; r < kR; ++r) {
+      const float p = ph[r];
+      const float* row = rows_s + r * S::RS + d_o;
+#pragma unroll
+      for (int i = 0; i < OPT; ++i) acc[i] = fmaf(p, row[i * TPH], acc[i]);
+    }
+  }
+  __syncthreads();
+  const float l = l_s[h_o];
+  const float inv = l > 0.0f ? 1.0f / l : 0.0f;
+  uint16_t* og = out + (qi * HA + h_o) * DD + d_o;
+#pragma unroll
+  for (int i = 0; i < OPT; ++i) {
+    __nv_bfloat16 v = __float2bfloat16_rn(acc[i] * inv);
+    og[i * TPH] = *reinterpret_cast<uint16_t*>(&v);
+  }
+  if (lse && d_o == 0) lse[qi * HA + h_o] = l > 0.0f ? m_s[h_o] + logf(l) : -INFINITY;
+}
+
+template <int HA, int DD>
+csa2_status run_simt(const void* q, const csa2_kv& kv, const int32_t* topk, int B, int Q, int k,
+                     float scale, void* out, float* lse, cudaStream_t stream) {
+  const size_t smem = AttnSmem<HA, DD>::bytes;
+  auto kern = kv.fmt == CSA2_KV_FP4 ? attn_simt_kernel<HA, DD, true> : attn_simt_kernel<HA, DD, false>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(smem)) != cudaSuccess)
+    return check_launch("sparse_attn: shared-memory opt-in");
+  if (B > 65535) return fail(CSA2_ERR_UNSUPPORTED, "sparse_attn: B > 65535");
+  kern<<<dim3(static_cast<unsigned>(Q), static_cast<unsigned>(B)), kT, smem, stream>>>(
+      static_cast<const uint16_t*>(q), kv.data, kv.scales, kv.n, topk, k, scale,
+      static_cast<uint16_t*>(out), lse, device_error_word());
+  note_launch(LK_ATTN);
+  return check_launch("sparse_attn");
+}
+
+}  // namespace
+
+size_t sparse_attn_workspace(int B, int Q, int Ha, int D, int k, csa2_kv_fmt fmt) {
+  return sparse_attn_tc_workspace(B, Q, Ha, D, k, fmt);
+}
+
+csa2_status launch_sparse_attn(const void* q, const csa2_kv& kv, const int32_t* topk, int B,
+                               int Q, int Ha, int k, float scale, void* out, float* lse, void* ws,
+                               size_t ws_bytes, cudaStream_t stream) {
+  if (B == 0 || Q == 0) return CSA2_OK;
+  csa2_status s = launch_sparse_attn_tc(q, kv, topk, B, Q, Ha, k, scale, out, lse, ws, ws_bytes,
+                                        stream);
+  if (s != CSA2_ERR_UNSUPPORTED) return s;
+  const int D = kv.dim;
+  if (Ha == 64 && D == 512) return run_simt<64, 512>(q, kv, topk, B, Q, k, scale, out, lse, stream);
+  if (Ha == 16 && D == 128) return run_simt<16, 128>(q, kv, topk, B, Q, k, scale, out, lse, stream);
+  if (Ha == 16 && D == 512) return run_simt<16, 512>(q, kv, topk, B, Q, k, scale, out, lse, stream);
+  if (Ha == 64 && D == 128) return run_simt<64, 128>(q, kv, topk, B, Q, k, scale, out, lse, stream);
+  if (Ha == 32 && D == 128) return run_simt<32, 128>(q, kv, topk, B, Q, k, scale, out, lse, stream);
+  if (Ha == 32 && D == 512) return run_simt<32, 512>(q, kv, topk, B, Q, k, scale, out, lse, stream);
+  return fail(CSA2_ERR_UNSUPPORTED, "sparse_attn: (Ha=%d, D=%d) not instantiated", Ha, D);
+}
+
+}  // namespace csa2

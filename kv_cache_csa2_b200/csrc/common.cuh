@@ -1,0 +1,63 @@
+// Shared internals of libcsa2: status plumbing, the per-device error word,
+// launch counters and small device helpers.  Not part of the C ABI.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "csa2.h"
+
+namespace csa2 {
+
+// ---------------------------------------------------------------- host side
+enum LaunchKind {
+  LK_COMPRESS = 0,
+  LK_INDEX = 1,
+  LK_TOPK = 2,
+  LK_ATTN = 3,
+  LK_COMBINE = 4,
+  LK_PACK = 5,
+  LK_UNPACK = 6,
+  LK_OTHER = 7,
+  LK_NUM = 8
+};
+void note_launch(LaunchKind kind, int n = 1);
+
+// Sets the thread-local message and returns `s`.
+csa2_status fail(csa2_status s, const char* fmt, ...);
+// CSA2_OK, or CSA2_ERR_CUDA with the pending launch error as the message.
+csa2_status check_launch(const char* what);
+// Host-side fault injection: returns the injected status or CSA2_OK.
+csa2_status fault_gate();
+// Device address of the current device's error word (resolved once per device).
+int* device_error_word();
+// Number of SMs of the current device (cached per device).
+int sm_count();
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+#define CSA2_TRY(expr)                          \
+  do {                                          \
+    csa2_status _s = (expr);                    \
+    if (_s != CSA2_OK) return _s;               \
+  } while (0)
+
+// -------------------------------------------------------------- device side
+enum : int { DEVERR_BOUNDS = CSA2_ERR_BOUNDS, DEVERR_TIMEOUT = CSA2_ERR_TIMEOUT };
+
+__device__ __forceinline__ void raise_dev_error(int* word, int code) {
+  if (word) atomicCAS(word, 0, code);
+}
+
+// bf16 halves of a 32-bit word -> f32 (exact)
+__device__ __forceinline__ float bf16_lo(uint32_t v) { return __uint_as_float(v << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t v) { return __uint_as_float(v & 0xffff0000u); }
+
+// f32 pair -> packed bf16x2, round to nearest even
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&h);
+}
+
+}  // namespace csa2

@@ -1,0 +1,33 @@
+// Internal launchers, one per kernel family.  Arguments are already validated
+// by the C-ABI layer (api.cu); each launcher picks the kernel instance and
+// enqueues it on `stream`.
+#pragma once
+
+#include "common.cuh"
+
+namespace csa2 {
+
+csa2_status launch_compress(const void* c, const float* z, const float* bias, int B, int64_t T,
+                            int D, int m, int halo, void* out, int64_t out_bstride,
+                            cudaStream_t stream);
+
+csa2_status launch_index_scores(const void* q, const float* w, const void* k, int B, int Q, int H,
+                                int d, int64_t N, const int32_t* n_visible, const int32_t* pool,
+                                int P, csa2_index_act act, float* scores, cudaStream_t stream);
+
+size_t select_topk_workspace(int64_t rows, int64_t L, int count);
+csa2_status launch_select_topk(const float* scores, int64_t rows, int64_t L, int count,
+                               const int32_t* ids, int32_t* out, void* ws, size_t ws_bytes,
+                               cudaStream_t stream);
+
+size_t sparse_attn_workspace(int B, int Q, int Ha, int D, int k, csa2_kv_fmt fmt);
+csa2_status launch_sparse_attn(const void* q, const csa2_kv& kv, const int32_t* topk, int B,
+                               int Q, int Ha, int k, float scale, void* out, float* lse, void* ws,
+                               size_t ws_bytes, cudaStream_t stream);
+
+csa2_status launch_fp4_pack(const void* x, int64_t rows, int D, uint8_t* codes, uint8_t* scales,
+                            cudaStream_t stream);
+csa2_status launch_fp4_unpack(const uint8_t* codes, const uint8_t* scales, int64_t rows, int D,
+                              void* x, cudaStream_t stream);
+
+}  // namespace csa2

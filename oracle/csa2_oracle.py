@@ -152,12 +152,12 @@ def index_scores(q: np.ndarray, w: np.ndarray, k: np.ndarray,
     """
     q = np.asarray(q, dtype=np.float64)
     w = np.asarray(w, dtype=np.float64)
-    k = np.asarray(k, dtype=np.float64)
     B, Q, H, d = q.shape
     N = k.shape[1]
     L = N if pool is None else pool.shape[2]
     out = np.full((B, Q, L), -np.inf, dtype=np.float64)
     for b in range(B):
+        kb = np.asarray(k[b], dtype=np.float64)      # one sequence at a time
         for t in range(Q):
             if pool is None:
                 ids = np.arange(N)
@@ -166,7 +166,7 @@ def index_scores(q: np.ndarray, w: np.ndarray, k: np.ndarray,
             else:
                 ids = np.asarray(pool[b, t], dtype=np.int64)
                 valid = ids >= 0
-            rows = k[b][np.where(valid, ids, 0)]          # [L, d]
+            rows = kb if pool is None else kb[np.where(valid, ids, 0)]   # [L, d]
             head_dots = rows @ q[b, t].T                  # [L, H]: q_h . k_j
             if act == "relu":
                 head_dots = np.maximum(head_dots, 0.0)
@@ -236,12 +236,14 @@ def sparse_attn(q: np.ndarray, kv: np.ndarray, topk: np.ndarray, scale: float):
     out[h] = sum_{j in S} softmax_j(scale * q[h] . kv[j]) * kv[j]
     lse[h] = log sum_{j in S} exp(scale * q[h] . kv[j])
 
-    Args: q [B, Q, Ha, D], kv [B, N, D] (values), topk [B, Q, k] entry ids
-    (-1 = empty).  An empty selection gives out = 0 and lse = -inf.
+    Args: q [B, Q, Ha, D]; kv [B, N, D] values, or a function kv(b, ids)
+    returning the float64 rows ids of sequence b (so a 1M-entry cache need not
+    be held in float64); topk [B, Q, k] entry ids (-1 = empty).  An empty
+    selection gives out = 0 and lse = -inf.
     Returns (o_exact [B,Q,Ha,D], o_bf16, lse [B,Q,Ha]) as float64.
     """
     q = np.asarray(q, dtype=np.float64)
-    kv = np.asarray(kv, dtype=np.float64)
+    rows_of = kv if callable(kv) else (lambda b, ids: np.asarray(kv[b][ids], dtype=np.float64))
     B, Q, Ha, D = q.shape
     o = np.zeros((B, Q, Ha, D), dtype=np.float64)
     lse = np.full((B, Q, Ha), -np.inf, dtype=np.float64)
@@ -251,7 +253,7 @@ def sparse_attn(q: np.ndarray, kv: np.ndarray, topk: np.ndarray, scale: float):
             ids = ids[ids >= 0]
             if ids.size == 0:
                 continue
-            ent = kv[b][ids]                          # [k', D]
+            ent = rows_of(b, ids)                     # [k', D]
             logits = scale * (q[b, t] @ ent.T)        # [Ha, k']
             top = logits.max(axis=1, keepdims=True)
             p = np.exp(logits - top)
@@ -373,8 +375,8 @@ def run_group(modes, layers, kv, index_k, k_top: int, scale: float,
                visible entry; keep a fresh top-k; attend.
     * reuse:   run no indexer; attend with the most recent selection.
 
-    kv: [B, N, D] main-KV values (already dequantised when stored as FP4);
-    index_k: [B, N, d].  layers[i] holds 'q_attn' and, for full/reindex,
+    kv: [B, N, D] main-KV values (already dequantised when stored as FP4), or
+    a row-fetch function kv(b, ids) as sparse_attn takes; index_k: [B, N, d].  layers[i] holds 'q_attn' and, for full/reindex,
     'q_index' and 'w_index'.  Returns a list of per-layer dicts with
     'topk', 'pool' (full only), 'o' (exact), 'o_bf16', 'lse'.
     """
