@@ -335,8 +335,14 @@ def fp4_pack(x: np.ndarray):
     blk = x.reshape(R, D // FP4_BLOCK, FP4_BLOCK)
     amax = np.abs(blk).max(axis=-1)                      # [R, D/16]
     scode = _nearest_code(amax, 6.0 * _E4M3_POS)         # 0..126
+    # Saturation: at or past the largest finite value the nearest is that value.
+    # (Stated explicitly because for huge inputs the float64 distances above all
+    # round to the same number and would look like a tie.)
+    scode = np.where(amax >= 6.0 * _E4M3_POS[-1], len(_E4M3_POS) - 1, scode)
     s = _E4M3_POS[scode]
-    mag_code = _nearest_code(np.abs(blk), _E2M1_MAGS[None, None, :] * s[..., None, None])
+    ax = np.abs(blk)
+    mag_code = _nearest_code(ax, _E2M1_MAGS[None, None, :] * s[..., None, None])
+    mag_code = np.where(ax >= 6.0 * s[..., None], 7, mag_code)
     mag_code = np.where(s[..., None] == 0.0, 0, mag_code)
     sign = np.signbit(blk).astype(np.int64) << 3
     code = (mag_code | sign).reshape(R, D)

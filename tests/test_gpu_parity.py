@@ -253,7 +253,7 @@ def _small(wl, **kw):
 
 
 SMALL = [
-    _small(C.C1, L=8192 // 4),
+    _small(C.C1, L=2048, compress_new_tokens=2048),
     _small(C.C2, B=3, L=4 * 3000, k=300),
     _small(C.C3, B=3, L=4 * 4000, k=100),
     _small(C.C4, B=2, L=4 * 20000, P=3000, k=500),

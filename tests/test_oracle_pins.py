@@ -327,6 +327,19 @@ def test_fp4_round_trips():
     assert np.array_equal(c2, codes) and np.array_equal(s2, scales)
 
 
+def test_fp4_saturation_for_huge_values():
+    # far past the top of both formats: scale 448 (0x7E), every code at +-6
+    x = np.zeros((3, 16))
+    x[0, :] = 1e30
+    x[1, :] = -3e38
+    x[2, 0], x[2, 1], x[2, 2] = 2700.0, -2688.0 * 1e6, 1.0
+    c, s = O.fp4_pack(x)
+    assert s.tolist() == [[0x7E], [0x7E], [0x7E]]
+    assert c[0].tolist() == [0x77] * 8 and c[1].tolist() == [0xFF] * 8
+    assert c[2, 0] == 0xF7            # 2700/448 > 6 -> 7; -2.688e9 -> -6 (0xF)
+    assert (c[2, 1] & 0xF) == 0       # 1/448 rounds to 0
+
+
 def test_fp4_zero_block():
     x = np.zeros((2, 32))
     x[1, 16:] = -0.0
