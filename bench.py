@@ -1,0 +1,531 @@
+#!/usr/bin/env python
+"""CSA2 layer-group benchmark on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config 4] [--impl ours|reference]
+
+A step is one pass of the layer group of the chosen workload (default: the
+1M-context hierarchical decode group, F + 3 Reindex + 4 Reuse, batch 8) over
+one batch of queries, with the KV cache and indexer keys resident in HBM.
+
+Timing (ours): every layer runs after an L2 flush (a 2x-L2 write outside the
+layer's event window, standing in for the FFN/MoE weights that stream between
+attention layers); a step's time is the sum of its per-layer CUDA-event times.
+`value` = queries of all ranks / max over ranks of that time.  Also reported:
+the same group back to back without flushes ("warm"), an end-to-end number
+through the public API with pinned host buffers and the copies inside the
+timed region ("e2e"), the dominant kernel's roofline from live per-kernel
+event timing, the SM clocks sampled during the timed region, and the CPU
+oracle on a bounded sample ("cpu_baseline").
+
+--impl reference times the float64 CPU oracle on the same workload, one
+query's layer group per step, on rank 0 only.
+
+Multi-GPU (torchrun): every rank runs its own replica of the workload; the
+path has no data-path collective (sequences are independent).
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import os
+import re
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "CSA2 decode queries/s per layer group at 1M ctx; achieved HBM TB/s vs peak"
+UNIT = "queries/s"
+L2_BYTES = 126 * 2 ** 20
+FALLBACK_HBM_GBS = 6650.0
+
+
+# ---------------------------------------------------------------------------- ranks
+
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def dist_init(world, backend):
+    import torch.distributed as dist
+    if world > 1 and not dist.is_initialized():
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=300))
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def reduce_max(x: float, world: int, device=None) -> float:
+    """Max of a float over all ranks (identity with one rank)."""
+    if world == 1:
+        return float(x)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ---------------------------------------------------------------------------- clocks
+
+CLOCK_FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,utilization.gpu,clocks_event_reasons.active,"
+                "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+                "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+REASON_COLS = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+
+
+class ClockSampler:
+    """nvidia-smi sampling every 200 ms while the timed region runs."""
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={CLOCK_FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+            time.sleep(0.3)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        rows = []
+        for line in open(self.path):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 10:
+                continue
+            try:
+                rows.append({"sm": float(parts[1]), "max": float(parts[2]), "util": float(parts[4]),
+                             "reasons": {c: ("Not" not in parts[6 + i]) for i, c in enumerate(REASON_COLS)}})
+            except ValueError:
+                continue
+        os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        load = [r for r in rows if r["util"] > 0] or rows
+        reasons = sorted({c for r in load for c, on in r["reasons"].items() if on})
+        return {"sm_mhz": statistics.median(r["sm"] for r in load),
+                "sm_max_mhz": max(r["max"] for r in rows), "reasons": reasons,
+                "samples": len(rows), "samples_under_load": len(load)}
+
+
+# ---------------------------------------------------------------------------- peaks, traffic
+
+def measured_hbm_gbs():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured"
+    except (OSError, KeyError, ValueError):
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def source_digest(*names) -> str:
+    h = hashlib.sha256()
+    for n in names:
+        with open(os.path.join(ROOT, "kv_cache_csa2_b200", "csrc", n), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:12]
+
+
+# kernel kind -> (source files whose digest must match the profile, profile summary)
+PROFILED_SOURCES = {
+    "index_scores": (("index_scores.cu", "index_scores_tc.cu"), "profiles/index_scores_c4.md"),
+    "attn": (("attn.cu", "attn_tc.cu"), "profiles/attn_c4.md"),
+    "topk": (("topk.cu", "topk_multi.cu"), "profiles/topk_c4.md"),
+}
+
+
+def ncu_traffic(kind):
+    """DRAM bytes per launch for `kind` from the committed ncu summary, or None
+    when there is none or the kernel source changed since it was taken."""
+    if kind not in PROFILED_SOURCES:
+        return None
+    srcs, path = PROFILED_SOURCES[kind]
+    try:
+        text = open(os.path.join(ROOT, path)).read()
+    except OSError:
+        return None
+    m = re.search(r"traffic_bytes_per_launch:\s*([0-9.eE+]+)\s+source_digest:\s*([0-9a-f]+)", text)
+    if not m or m.group(2) != source_digest(*srcs):
+        return None
+    return float(m.group(1))
+
+
+# ---------------------------------------------------------------------------- algorithmic bytes
+
+def algorithmic_bytes(wl):
+    """Bytes the method must move in one step, per kernel kind: the inputs it
+    has to read and the outputs it has to write (indexer keys of the scored
+    entries, gathered KV rows, q / w / out / lse / top-k / pool).  Score
+    intermediates are not counted.  Returns {kind: (bytes per step, launches
+    per step)}."""
+    rows = wl.B * wl.Q
+    qidx = rows * wl.Hi * (wl.d * 2 + 4)            # indexer q (bf16) + w (f32)
+    kv_row = wl.D * 2 if not wl.kv_fp4 else wl.D // 2 + wl.D // 16
+    out = {}
+    n_sel = sum(1 for m in wl.modes if m != "reuse")
+    n_full = sum(1 for m in wl.modes if m == "full")
+    n_re = n_sel - n_full
+    dense = n_full * (wl.B * wl.N * wl.d * 2 + qidx)
+    if n_re and wl.P == 0:
+        dense += n_re * (wl.B * wl.N * wl.d * 2 + qidx)
+    out["index_scores"] = (dense, n_full + (n_re if wl.P == 0 else 0))
+    if wl.P and n_re:
+        out["index_pool"] = (n_re * (rows * wl.P * (wl.d * 2 + 4) + qidx), n_re)
+    attn = wl.n_layers * (rows * wl.k * (kv_row + 4) + rows * wl.Ha * (wl.D * 2 * 2 + 4))
+    out["attn"] = (attn, wl.n_layers)
+    return out
+
+
+def kernel_min_bytes(wl):
+    """Per kind, what one launch of that kernel must at least move (for the
+    kernels whose inputs are intermediates, e.g. top-k reading the scores, this
+    is not part of the group's algorithmic bytes).  {kind: bytes per step}."""
+    rows = wl.B * wl.Q
+    alg = {k: v[0] for k, v in algorithmic_bytes(wl).items()}
+    n_full = sum(1 for m in wl.modes if m == "full")
+    n_re = sum(1 for m in wl.modes if m == "reindex")
+    L_full = wl.N
+    topk = n_full * rows * (L_full * 4 + (wl.k + wl.P) * 4) * (2 if wl.P else 1)
+    topk += n_re * rows * ((wl.P if wl.P else wl.N) * 4 + wl.k * 4)
+    alg["topk"] = topk
+    return alg
+
+
+# ---------------------------------------------------------------------------- ours
+
+def device_inputs(wl, inp, torch, device):
+    import numpy as np
+
+    def bf(bits):
+        return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).to(device)
+
+    d = {"kv": bf(inp["kv"]), "index_k": bf(inp["index_k"]),
+         "n_visible": torch.from_numpy(inp["n_visible"]).to(device) if inp["n_visible"] is not None else None,
+         "layers": []}
+    for L in inp["layers"]:
+        e = {"q_attn": bf(L["q_attn"])}
+        if "q_index" in L:
+            e["q_index"] = bf(L["q_index"])
+            e["w_index"] = torch.from_numpy(L["w_index"]).to(device)
+        d["layers"].append(e)
+    return d
+
+
+def run_ours(args, wl, world, rank, local):
+    import torch
+    import kv_cache_csa2_b200 as K
+    from kv_cache_csa2_b200 import inputs as I
+
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py: no CUDA device")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    dist_init(world, "nccl")
+    K.lib()
+    inp = I.make_inputs(wl, seed=args.seed)
+    D = device_inputs(wl, inp, torch, dev)
+    kv, kv_scales = D["kv"], None
+    if wl.kv_fp4:
+        kv, kv_scales = K.csa2_fp4_pack(D["kv"])
+    modes = [{"full": K.FULL, "reindex": K.REINDEX, "reuse": K.REUSE}[m] for m in wl.modes]
+    g = K.Group(wl.B, wl.Q, wl.N, wl.D, wl.Ha, wl.Hi, wl.d, wl.k, modes, P=wl.P, scale=wl.attn_scale,
+                kv_fmt=K.KV_FP4 if wl.kv_fp4 else K.KV_BF16)
+    outs = [torch.empty(wl.B, wl.Q, wl.Ha, wl.D, dtype=torch.bfloat16, device=dev) for _ in wl.modes]
+    lses = [torch.empty(wl.B, wl.Q, wl.Ha, dtype=torch.float32, device=dev) for _ in wl.modes]
+    kws = []
+    for i, mode in enumerate(wl.modes):
+        L = D["layers"][i]
+        kw = {}
+        if mode == "full":
+            kw = dict(kv=kv, kv_scales=kv_scales, index_k=D["index_k"], n_visible=D["n_visible"])
+        elif mode == "reindex":
+            kw = dict(n_visible=D["n_visible"])
+        if mode != "reuse":
+            kw.update(q_index=L["q_index"], w_index=L["w_index"])
+        kws.append(kw)
+
+    def layer(i):
+        g.layer(i, D["layers"][i]["q_attn"], outs[i], lses[i], **kws[i])
+
+    flush_buf = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device=dev)
+
+    def flush():
+        flush_buf.fill_(1.0)
+
+    n_layers = wl.n_layers
+    # ---- cold: flush before every layer, per-layer events
+    for _ in range(args.warmup):
+        for i in range(n_layers):
+            flush()
+            layer(i)
+    torch.cuda.synchronize()
+    K.csa2_device_error()
+    ev = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(n_layers)] for _ in range(args.steps)]
+    sampler = ClockSampler(local)
+    K.reset_launch_counts()
+    K.timing_reset()
+    barrier(world)
+    torch.cuda.synchronize()
+    sampler.start()
+    K.timing_enable(True)
+    t0 = time.perf_counter()
+    for s in range(args.steps):
+        for i in range(n_layers):
+            flush()
+            ev[s][i][0].record()
+            layer(i)
+            ev[s][i][1].record()
+    torch.cuda.synchronize()
+    barrier(world)
+    wall = time.perf_counter() - t0
+    K.timing_enable(False)
+    clocks = sampler.stop()
+    launches = K.launch_counts()
+    ktimes = K.kernel_times()
+    K.csa2_device_error()
+    step_ms = [sum(a.elapsed_time(b) for a, b in ev[s]) for s in range(args.steps)]
+    layer_ms = [statistics.mean(ev[s][i][0].elapsed_time(ev[s][i][1]) for s in range(args.steps))
+                for i in range(n_layers)]
+    ms_local = statistics.mean(step_ms)
+    ms = reduce_max(ms_local, world, dev)
+    queries = world * wl.B * wl.Q
+    value = queries / (ms / 1e3)
+
+    # ---- warm: the group back to back
+    for _ in range(args.warmup):
+        for i in range(n_layers):
+            layer(i)
+    barrier(world)
+    torch.cuda.synchronize()
+    w0, w1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    w0.record()
+    for _ in range(args.steps):
+        for i in range(n_layers):
+            layer(i)
+    w1.record()
+    torch.cuda.synchronize()
+    warm_ms = reduce_max(w0.elapsed_time(w1) / args.steps, world, dev)
+
+    # ---- e2e: host inputs -> API -> host outputs, copies inside the timed region
+    h_in, d_in = [], []
+    for i in range(n_layers):
+        for key in ("q_attn", "q_index", "w_index"):
+            t = D["layers"][i].get(key)
+            if t is not None:
+                h_in.append(t.cpu().pin_memory())
+                d_in.append(t)
+    h_out = [o.cpu().pin_memory() for o in outs] + [l.cpu().pin_memory() for l in lses]
+    d_out = outs + lses
+    bi = sum(t.numel() * t.element_size() for t in h_in)
+    bo = sum(t.numel() * t.element_size() for t in h_out)
+
+    def e2e_step():
+        for h, d in zip(h_in, d_in):
+            d.copy_(h, non_blocking=True)
+        for i in range(n_layers):
+            layer(i)
+        for h, d in zip(h_out, d_out):
+            h.copy_(d, non_blocking=True)
+
+    for _ in range(args.warmup):
+        e2e_step()
+    barrier(world)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(args.steps):
+        e2e_step()
+    e1.record()
+    torch.cuda.synchronize()
+    e2e_ms = reduce_max(e0.elapsed_time(e1) / args.steps, world, dev)
+    g.close()
+
+    # ---- roofline of the dominant kernel (largest device time in the cold region)
+    hbm, peak_src = measured_hbm_gbs()
+    alg = algorithmic_bytes(wl)
+    per_kind = {k: v for k, v in ktimes.items() if v[1] > 0}
+    dom = max(per_kind, key=lambda k: per_kind[k][0]) if per_kind else None
+    roof = None
+    if dom is not None:
+        tot_ms, n = per_kind[dom]
+        avg_s = tot_ms / n / 1e3
+        step_bytes = kernel_min_bytes(wl).get(dom, 0)
+        bytes_per_launch = step_bytes / max(n / args.steps, 1)
+        achieved = bytes_per_launch / avg_s / 1e9 if avg_s > 0 else 0.0
+        roof = {"kernel": dom, "bound": "hbm", "achieved": round(achieved, 1), "peak": hbm,
+                "unit": "GB/s", "frac": round(achieved / hbm, 4), "traffic": ncu_traffic(dom),
+                "algorithmic_bytes_per_launch": int(bytes_per_launch),
+                "avg_launch_us": round(avg_s * 1e6, 2), "launches": n,
+                "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs)" if peak_src == "measured"
+                else "fallback 6650 GB/s"}
+    kernels = {k: {"total_ms": round(v[0], 4), "launches": v[1],
+                   "avg_us": round(v[0] / v[1] * 1e3, 2)} for k, v in per_kind.items()}
+    total_alg = sum(v[0] for v in alg.values())
+    res = {
+        "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded N(0,1)/U(0,1) inputs of the workload's shapes)",
+        "config": {"workload": wl.name, "B": wl.B, "Q": wl.Q, "L": wl.L, "m": wl.m, "N": wl.N,
+                   "D": wl.D, "Ha": wl.Ha, "Hi": wl.Hi, "d": wl.d, "k": wl.k, "P": wl.P,
+                   "modes": ",".join(wl.modes), "kv": "fp4" if wl.kv_fp4 else "bf16",
+                   "l2": "flushed before every layer (2x L2 write outside the layer's events); "
+                         "ms_per_step = sum of per-layer CUDA-event times",
+                   "parallelism": f"replicas x{world}"},
+        "group_bytes": int(total_alg),
+        "group_achieved_gbs": round(total_alg / (ms_local / 1e3) / 1e9, 1),
+        "group_frac_of_hbm": round(total_alg / (ms_local / 1e3) / 1e9 / hbm, 4),
+        "layer_ms": [round(x, 4) for x in layer_ms],
+        "warm": {"ms_per_step": round(warm_ms, 4), "value": round(queries / (warm_ms / 1e3), 1),
+                 "note": "same group back to back, no L2 flush"},
+        "e2e": {"value": round(queries / (e2e_ms / 1e3), 1), "unit": UNIT,
+                "h2d_bytes_per_step": bi, "d2h_bytes_per_step": bo,
+                "note": "per step: pinned-host -> device copy of every layer's queries and head "
+                        "weights, the group through the C ABI, device -> pinned-host copy of every "
+                        "layer's output and lse; KV cache and indexer keys stay resident"},
+        "roofline": roof,
+        "kernels": kernels,
+        "gpu_launches": int(sum(launches.values())),
+        "clocks": clocks,
+        "wall_s_timed_region": round(wall, 4),
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        res["cpu_baseline"] = cpu_baseline(wl, inp, budget_s=args.cpu_budget)
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+        dist.destroy_process_group()
+    return res
+
+
+# ---------------------------------------------------------------------------- oracle (CPU)
+
+def oracle_queries(wl, inp, queries):
+    """Run the oracle's layer group for the listed (b, q) queries; returns seconds."""
+    import numpy as np
+    import oracle as O
+    from kv_cache_csa2_b200 import inputs as I
+
+    t0 = time.perf_counter()
+    for b, t in queries:
+        kb = inp["kv"][b:b + 1]
+
+        def rows(_, ids, kb=kb):
+            r = O.bf16_bits_to_float(kb[0, ids])
+            return O.fp4_unpack(*O.fp4_pack(r)) if wl.kv_fp4 else r
+
+        layers = []
+        for L in inp["layers"]:
+            d = {"q_attn": O.bf16_bits_to_float(L["q_attn"][b:b + 1, t:t + 1])}
+            if "q_index" in L:
+                d["q_index"] = O.bf16_bits_to_float(L["q_index"][b:b + 1, t:t + 1])
+                d["w_index"] = L["w_index"][b:b + 1, t:t + 1].astype(np.float64)
+            layers.append(d)
+        nv = inp["n_visible"][b:b + 1, t:t + 1] if inp["n_visible"] is not None else None
+        O.run_group(list(wl.modes), layers, rows, I.bf16_bits_to_f32(inp["index_k"][b:b + 1]), wl.k,
+                    wl.attn_scale, pool_size=wl.P, n_visible=nv)
+    return time.perf_counter() - t0
+
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        return max((i.get("num_threads", 1) for i in threadpool_info()), default=1)
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def cpu_baseline(wl, inp, budget_s=20.0):
+    qs = [(b, t) for b in range(wl.B) for t in range(wl.Q)]
+    done, spent = 0, 0.0
+    while done < len(qs) and spent < budget_s:
+        spent += oracle_queries(wl, inp, [qs[done]])
+        done += 1
+    return {"value": round(done / spent, 3), "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+            "sample": f"{done} of the workload's {len(qs)} queries, each through the whole layer group "
+                      f"(float64 numpy oracle), {spent:.1f} s"}
+
+
+def run_reference(args, wl, world, rank):
+    if rank != 0:
+        return None
+    from kv_cache_csa2_b200 import inputs as I
+    inp = I.make_inputs(wl, seed=args.seed)
+    qs = [(b, t) for b in range(wl.B) for t in range(wl.Q)]
+    for i in range(args.warmup):
+        oracle_queries(wl, inp, [qs[i % len(qs)]])
+    spent = 0.0
+    for i in range(args.steps):
+        spent += oracle_queries(wl, inp, [qs[i % len(qs)]])
+    value = args.steps / spent
+    cores = blas_threads()
+    sample = f"{args.steps} single-query layer groups of the workload (float64 numpy oracle)"
+    return {"impl": "reference", "metric": METRIC, "value": round(value, 3), "unit": UNIT,
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(spent / args.steps * 1e3, 3), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic (seeded N(0,1)/U(0,1) inputs of the workload's shapes)",
+            "config": {"workload": wl.name, "B": wl.B, "Q": wl.Q, "L": wl.L, "N": wl.N, "D": wl.D,
+                       "k": wl.k, "P": wl.P, "modes": ",".join(wl.modes),
+                       "sample_per_step": "one query"},
+            "cpu_baseline": {"value": round(value, 3), "unit": UNIT, "cores": cores,
+                             "kind": "oracle", "sample": sample},
+            "e2e": {"value": round(value, 3), "unit": UNIT, "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+
+
+# ---------------------------------------------------------------------------- main
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.split("\n\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--config", type=int, default=4, choices=[1, 2, 3, 4, 5])
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--cpu-budget", type=float, default=20.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    from kv_cache_csa2_b200.configs import CONFIGS
+    wl = CONFIGS[args.config]
+    world, rank, local = dist_env()
+    if args.impl == "reference":
+        res = run_reference(args, wl, world, rank)
+    else:
+        res = run_ours(args, wl, world, rank, local)
+    if rank == 0 and res is not None:
+        print(json.dumps(res), flush=True)
+
+
+if __name__ == "__main__":
+    main()

@@ -262,10 +262,20 @@ const char* csa2_last_error(void);
  * CSA2_ERR_TIMEOUT) and clears it. */
 csa2_status csa2_device_error(csa2_stream stream);
 /* Kernel launches issued by this library since the last reset, per kind:
- * 0 compress, 1 index scores, 2 top-k, 3 attention, 4 attention combine,
- * 5 fp4 pack, 6 fp4 unpack, 7 other (memsets).  Returns the number of kinds. */
+ * 0 compress, 1 index scores (all entries), 2 top-k, 3 attention, 4 attention
+ * combine, 5 fp4 pack, 6 fp4 unpack, 7 other (memsets), 8 index scores inside
+ * a pool.  Returns the number of kinds. */
 int csa2_launch_counts(int64_t* counts, int n);
 void csa2_reset_launch_counts(void);
+/* Per-kind device time of this library's kernels (instrumentation).  While
+ * enabled, each launch is bracketed by two CUDA events recorded on its own
+ * stream (not inside stream capture).  csa2_kernel_times() waits for the
+ * recorded events and returns, for each kind (numbered as above), the summed
+ * milliseconds and the number of timed launches since the last reset; it
+ * returns the number of kinds. */
+csa2_status csa2_timing_enable(int on);
+int csa2_kernel_times(double* ms, int64_t* launches, int n);
+void csa2_timing_reset(void);
 /* Host-side fault injection for tests: "alloc", "launch" or "" (off).  While
  * set, every call returns CSA2_ERR_OOM / CSA2_ERR_CUDA before touching the
  * device.  The environment variable CSA2_FAULT sets the initial value. */

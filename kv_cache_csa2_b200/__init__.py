@@ -66,6 +66,9 @@ _SIGS = {
     "csa2_launch_counts": (_I, [ctypes.POINTER(_I64), _I]),
     "csa2_reset_launch_counts": (None, []),
     "csa2_set_fault": (_I, [ctypes.c_char_p]),
+    "csa2_timing_enable": (_I, [_I]),
+    "csa2_kernel_times": (_I, [ctypes.POINTER(ctypes.c_double), ctypes.POINTER(_I64), _I]),
+    "csa2_timing_reset": (None, []),
     "csa2_version": (_I, []),
 }
 EXPORTED_SYMBOLS = tuple(_SIGS)
@@ -317,7 +320,7 @@ def csa2_device_error(stream=None):
 
 
 LAUNCH_KINDS = ("compress", "index_scores", "topk", "attn", "attn_combine", "fp4_pack",
-                "fp4_unpack", "other")
+                "fp4_unpack", "other", "index_pool")
 
 
 def launch_counts() -> dict:
@@ -328,6 +331,24 @@ def launch_counts() -> dict:
 
 def reset_launch_counts() -> None:
     lib().csa2_reset_launch_counts()
+
+
+def timing_enable(on: bool) -> None:
+    """Bracket every library launch with CUDA events (instrumentation)."""
+    _check(lib().csa2_timing_enable(int(bool(on))))
+
+
+def timing_reset() -> None:
+    lib().csa2_timing_reset()
+
+
+def kernel_times() -> dict:
+    """{kind: (total_ms, timed_launches)} since the last timing_reset()."""
+    n = len(LAUNCH_KINDS)
+    ms = (ctypes.c_double * n)()
+    cnt = (_I64 * n)()
+    lib().csa2_kernel_times(ms, cnt, n)
+    return {k: (ms[i], cnt[i]) for i, k in enumerate(LAUNCH_KINDS)}
 
 
 def set_fault(kind: str) -> None:

@@ -8,6 +8,7 @@
 #include <cstdlib>
 #include <cstring>
 #include <mutex>
+#include <vector>
 
 #include "common.cuh"
 #include "launchers.h"
@@ -56,7 +57,60 @@ csa2_status fault_gate() {
 // ---------------------------------------------------------- launch counters
 static std::atomic<long long> g_launches[LK_NUM];
 
-void note_launch(LaunchKind kind, int n) { g_launches[kind] += n; }
+// -------------------------------------------------------- launch timing
+struct TimedLaunch {
+  int kind;
+  cudaEvent_t start, stop;
+};
+static std::atomic<bool> g_timing{false};
+static std::mutex g_tmu;
+static std::vector<cudaEvent_t> g_event_pool;
+static std::vector<TimedLaunch> g_timed;
+static double g_ms[LK_NUM];
+static long long g_timed_n[LK_NUM];
+static thread_local cudaEvent_t t_start = nullptr;
+
+static cudaEvent_t take_event() {
+  std::lock_guard<std::mutex> lk(g_tmu);
+  if (!g_event_pool.empty()) {
+    cudaEvent_t e = g_event_pool.back();
+    g_event_pool.pop_back();
+    return e;
+  }
+  cudaEvent_t e = nullptr;
+  if (cudaEventCreate(&e) != cudaSuccess) {
+    cudaGetLastError();
+    return nullptr;
+  }
+  return e;
+}
+
+static bool capturing(cudaStream_t s) {
+  cudaStreamCaptureStatus st = cudaStreamCaptureStatusNone;
+  if (cudaStreamIsCapturing(s, &st) != cudaSuccess) {
+    cudaGetLastError();
+    return true;
+  }
+  return st != cudaStreamCaptureStatusNone;
+}
+
+void begin_launch(cudaStream_t s) {
+  if (!g_timing.load(std::memory_order_relaxed) || capturing(s)) return;
+  t_start = take_event();
+  if (t_start) cudaEventRecord(t_start, s);
+}
+
+void note_launch(LaunchKind kind, int n, cudaStream_t s) {
+  g_launches[kind] += n;
+  if (!t_start) return;
+  cudaEvent_t stop = take_event();
+  if (stop) {
+    cudaEventRecord(stop, s);
+    std::lock_guard<std::mutex> lk(g_tmu);
+    g_timed.push_back({static_cast<int>(kind), t_start, stop});
+  }
+  t_start = nullptr;
+}
 
 // ------------------------------------------------------- device error word
 __device__ int g_dev_err;
@@ -142,6 +196,48 @@ int csa2_launch_counts(int64_t* counts, int n) {
 
 void csa2_reset_launch_counts(void) {
   for (int i = 0; i < LK_NUM; ++i) g_launches[i] = 0;
+}
+
+csa2_status csa2_timing_enable(int on) {
+  g_timing.store(on != 0);
+  return CSA2_OK;
+}
+
+int csa2_kernel_times(double* ms, int64_t* launches, int n) {
+  std::vector<TimedLaunch> pending;
+  {
+    std::lock_guard<std::mutex> lk(g_tmu);
+    pending.swap(g_timed);
+  }
+  for (const TimedLaunch& t : pending) {
+    float f = 0.0f;
+    if (cudaEventSynchronize(t.stop) == cudaSuccess &&
+        cudaEventElapsedTime(&f, t.start, t.stop) == cudaSuccess) {
+      std::lock_guard<std::mutex> lk(g_tmu);
+      g_ms[t.kind] += f;
+      g_timed_n[t.kind] += 1;
+    } else {
+      cudaGetLastError();
+    }
+    std::lock_guard<std::mutex> lk(g_tmu);
+    g_event_pool.push_back(t.start);
+    g_event_pool.push_back(t.stop);
+  }
+  std::lock_guard<std::mutex> lk(g_tmu);
+  for (int i = 0; i < n && i < LK_NUM; ++i) {
+    if (ms) ms[i] = g_ms[i];
+    if (launches) launches[i] = g_timed_n[i];
+  }
+  return LK_NUM;
+}
+
+void csa2_timing_reset(void) {
+  csa2_kernel_times(nullptr, nullptr, 0);   // drain what is pending
+  std::lock_guard<std::mutex> lk(g_tmu);
+  for (int i = 0; i < LK_NUM; ++i) {
+    g_ms[i] = 0.0;
+    g_timed_n[i] = 0;
+  }
 }
 
 csa2_status csa2_device_error(csa2_stream stream) {

@@ -190,10 +190,11 @@ csa2_status run_simt(const void* q, const csa2_kv& kv, const int32_t* topk, int 
                            static_cast<int>(smem)) != cudaSuccess)
     return check_launch("sparse_attn: shared-memory opt-in");
   if (B > 65535) return fail(CSA2_ERR_UNSUPPORTED, "sparse_attn: B > 65535");
+  begin_launch(stream);
   kern<<<dim3(static_cast<unsigned>(Q), static_cast<unsigned>(B)), kT, smem, stream>>>(
       static_cast<const uint16_t*>(q), kv.data, kv.scales, kv.n, topk, k, scale,
       static_cast<uint16_t*>(out), lse, device_error_word());
-  note_launch(LK_ATTN);
+  note_launch(LK_ATTN, 1, stream);
   return check_launch("sparse_attn");
 }
 

@@ -20,9 +20,14 @@ enum LaunchKind {
   LK_PACK = 5,
   LK_UNPACK = 6,
   LK_OTHER = 7,
-  LK_NUM = 8
+  LK_INDEX_POOL = 8,
+  LK_NUM = 9
 };
-void note_launch(LaunchKind kind, int n = 1);
+// Call begin_launch(stream) right before a kernel launch and
+// note_launch(kind, n, stream) right after it: counts the launch and, when
+// timing is enabled, brackets it with events on `stream`.
+void begin_launch(cudaStream_t stream);
+void note_launch(LaunchKind kind, int n = 1, cudaStream_t stream = nullptr);
 
 // Sets the thread-local message and returns `s`.
 csa2_status fail(csa2_status s, const char* fmt, ...);

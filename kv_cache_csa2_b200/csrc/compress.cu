@@ -86,10 +86,11 @@ csa2_status launch_compress(const void* c, const float* z, const float* bias, in
   const int64_t work = N * (D / 8);
   const int threads = 256;
   dim3 grid(static_cast<unsigned>((work + threads - 1) / threads), static_cast<unsigned>(B));
+  begin_launch(stream);
   compress_kernel<<<grid, threads, 0, stream>>>(
       static_cast<const uint16_t*>(c), z, bias, static_cast<int>(N), D, m, halo ? m : 0, t_in,
       static_cast<uint16_t*>(out), out_bstride);
-  note_launch(LK_COMPRESS);
+  note_launch(LK_COMPRESS, 1, stream);
   return check_launch("compress");
 }
 

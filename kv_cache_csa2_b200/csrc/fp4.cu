@@ -122,9 +122,10 @@ csa2_status launch_fp4_pack(const void* x, int64_t rows, int D, uint8_t* codes, 
   if (nb == 0) return CSA2_OK;
   const int threads = 256;
   const int64_t grid = (nb + threads - 1) / threads;
+  begin_launch(stream);
   fp4_pack_kernel<<<static_cast<unsigned>(grid), threads, 0, stream>>>(
       static_cast<const uint4*>(x), nb, reinterpret_cast<uint2*>(codes), scales);
-  note_launch(LK_PACK);
+  note_launch(LK_PACK, 1, stream);
   return check_launch("fp4_pack");
 }
 
@@ -134,9 +135,10 @@ csa2_status launch_fp4_unpack(const uint8_t* codes, const uint8_t* scales, int64
   if (nb == 0) return CSA2_OK;
   const int threads = 256;
   const int64_t grid = (nb + threads - 1) / threads;
+  begin_launch(stream);
   fp4_unpack_kernel<<<static_cast<unsigned>(grid), threads, 0, stream>>>(
       reinterpret_cast<const uint2*>(codes), scales, nb, static_cast<uint4*>(x));
-  note_launch(LK_UNPACK);
+  note_launch(LK_UNPACK, 1, stream);
   return check_launch("fp4_unpack");
 }
 

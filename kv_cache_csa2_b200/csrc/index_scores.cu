@@ -101,10 +101,11 @@ csa2_status run_simt(const void* q, const float* w, const void* k, int B, int Q,
   }
   dim3 grid(static_cast<unsigned>((L + kThreads - 1) / kThreads), static_cast<unsigned>(Q),
             static_cast<unsigned>(B));
+  begin_launch(stream);
   kern<<<grid, kThreads, smem, stream>>>(
       static_cast<const uint16_t*>(q), w, static_cast<const uint16_t*>(k), Q, H, d, N, n_visible,
       pool, P, act == CSA2_ACT_RELU ? 1 : 0, scores, device_error_word());
-  note_launch(LK_INDEX);
+  note_launch(pool ? LK_INDEX_POOL : LK_INDEX, 1, stream);
   return check_launch("index_scores");
 }
 

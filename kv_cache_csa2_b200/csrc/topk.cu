@@ -164,8 +164,9 @@ csa2_status launch_select_topk(const float* scores, int64_t rows, int64_t L, int
   csa2_status s = launch_select_topk_multi(scores, rows, L, count, ids, out, ws, ws_bytes, stream);
   if (s != CSA2_ERR_UNSUPPORTED) return s;
   if (rows > 0x7fffffff) return fail(CSA2_ERR_UNSUPPORTED, "select_topk: too many rows");
+  begin_launch(stream);
   topk_row_kernel<<<static_cast<unsigned>(rows), kT, 0, stream>>>(scores, L, count, ids, out);
-  note_launch(LK_TOPK);
+  note_launch(LK_TOPK, 1, stream);
   return check_launch("select_topk");
 }
 
