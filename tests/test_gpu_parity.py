@@ -136,7 +136,9 @@ def _score_tol(q, w, k, pool=None):
 
 
 @pytest.mark.parametrize("B,Q,H,d,N", [(2, 3, 8, 64, 1000), (1, 2, 64, 128, 777), (2, 1, 16, 32, 300),
-                                       (1, 1, 128, 64, 129), (3, 2, 4, 256, 65)])
+                                       (1, 1, 128, 64, 129), (3, 2, 4, 256, 65),
+                                       (1, 37, 8, 64, 500), (2, 9, 64, 128, 300), (1, 6, 48, 64, 1300),
+                                       (3, 1, 64, 128, 128), (1, 1, 1, 128, 4000)])
 @pytest.mark.parametrize("act", [K.ACT_RELU, K.ACT_IDENTITY])
 def test_index_scores_parity(B, Q, H, d, N, act):
     r = _rng(5)
@@ -152,9 +154,10 @@ def test_index_scores_parity(B, Q, H, d, N, act):
     assert np.all(np.abs(got[fin] - want[fin]) <= tol[fin])
 
 
-def test_index_scores_pool_parity():
+@pytest.mark.parametrize("B,Q,H,d,N,P", [(2, 2, 64, 128, 5000, 700), (3, 1, 8, 64, 2000, 300),
+                                         (1, 3, 16, 128, 999, 129)])
+def test_index_scores_pool_parity(B, Q, H, d, N, P):
     r = _rng(6)
-    B, Q, H, d, N, P = 2, 2, 64, 128, 5000, 700
     q, w, k = _index_inputs(r, B, Q, H, d, N)
     pool = np.sort(r.choice(N, size=(B, Q, P)), axis=-1).astype(np.int32)
     pool[:, :, -13:] = -1
