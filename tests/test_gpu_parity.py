@@ -217,7 +217,9 @@ def _attn_case(r, B, Q, Ha, D, N, k, fp4):
 @pytest.mark.parametrize("Ha,D,N,k,fp4", [(16, 128, 3000, 256, False), (16, 128, 3000, 256, True),
                                           (64, 512, 5000, 2048, False), (64, 512, 900, 100, False),
                                           (64, 512, 5000, 2048, True), (16, 512, 500, 33, False),
-                                          (32, 128, 400, 17, True)])
+                                          (32, 128, 400, 17, True), (64, 512, 9000, 4096, False),
+                                          (64, 512, 9000, 6000, False), (64, 512, 2000, 300, False),
+                                          (64, 512, 3000, 129, False)])
 def test_sparse_attn_parity(Ha, D, N, k, fp4):
     r = _rng(9)
     B, Q = 2, 3
@@ -233,6 +235,19 @@ def test_sparse_attn_parity(Ha, D, N, k, fp4):
         kvv = O.bf16_bits_to_float(kv)
     o, _, l = O.sparse_attn(O.bf16_bits_to_float(q), kvv, topk, scale)
     U.check_attn(U.host_bf16(out), lse.cpu().numpy().astype(np.float64), o, l, f"Ha{Ha} D{D} k{k}")
+
+
+@pytest.mark.parametrize("max_cluster", ["1", "2", "4", "8"])
+def test_sparse_attn_smaller_clusters(max_cluster, monkeypatch):
+    """The tensor-core kernel splits a query over a cluster of CTAs; smaller
+    clusters give each CTA more tiles (re-gathered for the PV product)."""
+    monkeypatch.setenv("CSA2_ATTN_MAX_CLUSTER", max_cluster)
+    r = _rng(19)
+    B, Q, Ha, D, N, k = 2, 2, 64, 512, 4000, 384 if max_cluster == "1" else 1000
+    q, kv, topk = _attn_case(r, B, Q, Ha, D, N, k, False)
+    out, lse = K.csa2_sparse_attn(U.dev_bf16(q), U.dev_bf16(kv), U.dev(topk), D ** -0.5)
+    o, _, l = O.sparse_attn(O.bf16_bits_to_float(q), O.bf16_bits_to_float(kv), topk, D ** -0.5)
+    U.check_attn(U.host_bf16(out), lse.cpu().numpy().astype(np.float64), o, l, f"cluster<={max_cluster}")
 
 
 def test_sparse_attn_bounds_recorded_not_faulting():
