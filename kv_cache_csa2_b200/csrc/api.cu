@@ -366,6 +366,12 @@ csa2_status csa2_index_topk(csa2_mode mode, const void* q, const float* w, const
   const size_t sel_bytes = workspace_bytes - sbytes;
   CSA2_TRY(launch_index_scores(q, w, k, B, Q, H, d, N, n_visible, pool_in, pool_in ? P_in : 0, act,
                                scores, s));
+  if (pool_out) {
+    // the pool and the top-k in the same selection passes when the kernel applies
+    const csa2_status st = launch_select_topk2(scores, rows, L, k_top, nullptr, topk_out, P_out,
+                                               pool_out, sel_ws, sel_bytes, s);
+    if (st != CSA2_ERR_UNSUPPORTED) return st;
+  }
   CSA2_TRY(launch_select_topk(scores, rows, L, k_top, pool_in, topk_out, sel_ws, sel_bytes, s));
   if (pool_out)
     CSA2_TRY(launch_select_topk(scores, rows, L, P_out, nullptr, pool_out, sel_ws, sel_bytes, s));

@@ -34,8 +34,11 @@ using namespace sm100;
 
 constexpr int kWarps = 6;
 constexpr int kThreads = kWarps * 32;
+// pool scoring gathers rows with cp.async from four producer warps (0, 6, 7, 8)
+constexpr int kPoolThreads = 9 * 32;
 constexpr int kTileRows = 128;
 constexpr int kKBlockBytes = kTileRows * 128;  // 128 rows x 64 bf16
+constexpr int kLag = 2;                        // pool gathers: stages of copies kept in flight
 
 struct Params {
   const uint16_t* q;
@@ -76,7 +79,7 @@ struct Cfg {
 };
 
 template <int DK, int NQ, int HP, bool POOL>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(POOL ? kPoolThreads : kThreads, 1)
     index_tc_kernel(const __grid_constant__ CUtensorMap kmap, const Params p) {
   using C = Cfg<DK, NQ, HP, POOL>;
   constexpr int S = C::STAGES;
@@ -104,7 +107,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < S; ++i) {
-      mbar_init(&full[i], POOL ? 32 : 1);
+      mbar_init(&full[i], POOL ? kTileRows : 1);
       mbar_init(&empty[i], 1);
     }
     for (int i = 0; i < 2; ++i) {
@@ -126,8 +129,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
 
-  if (warp == 0) {
+  if (warp == 0 || (POOL && warp >= 6)) {
     // ---------------------------------------------------------------- producer
+    const int ptid = warp == 0 ? lane : 32 + (warp - 6) * 32 + lane;   // pool: row of the tile
     int64_t prev_bg = -1;
     int qi = -1;
     int64_t it = 0;
@@ -137,7 +141,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int t = static_cast<int>(u % p.n_tiles);
       const int b = static_cast<int>(bg / p.n_qgroups);
       const int g = static_cast<int>(bg % p.n_qgroups);
-      if (bg != prev_bg) {
+      if (bg != prev_bg && warp != 0) {
+        ++qi;
+        prev_bg = bg;
+      } else if (bg != prev_bg) {
         ++qi;
         const int slot = qi & 1;
         if (qi >= 2 && !mbar_wait(&qempty[slot], ((qi >> 1) - 1) & 1, abort_flag, p.err)) { ok = false; break; }
@@ -175,9 +182,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       } else {
         const int64_t qrow = static_cast<int64_t>(b) * p.Q + g;   // NQ == 1 for pools
-#pragma unroll
-        for (int rr = 0; rr < 4; ++rr) {
-          const int r = lane + 32 * rr;
+        {
+          const int r = ptid;                                     // one row per producer thread
           const int64_t slot_i = static_cast<int64_t>(t) * kTileRows + r;
           int64_t id = slot_i < L ? p.pool[qrow * p.P + slot_i] : -1;
           const bool valid = id >= 0 && id < p.N;
@@ -187,10 +193,18 @@ __global__ void __launch_bounds__(kThreads, 1)
             cp_async_16(dst + (c / 8) * kKBlockBytes + sw128_offset(r, c % 8), src + c * 8, valid ? 16u : 0u);
         }
         cp_async_commit();
-        cp_async_wait<0>();
-        fence_proxy_async_smem();
-        mbar_arrive(&full[stage]);
+        // keep kLag stages of copies in flight; stage it-kLag is complete now
+        if (it >= kLag) {
+          cp_async_wait<kLag>();
+          fence_proxy_async_smem();
+          mbar_arrive(&full[(it - kLag) % S]);
+        }
       }
+    }
+    if (POOL) {
+      cp_async_wait<0>();
+      fence_proxy_async_smem();
+      for (int64_t j = (it > kLag ? it - kLag : 0); j < it; ++j) mbar_arrive(&full[j % S]);
     }
     if (!ok && !POOL && lane == 0) {
       // let TMA loads still in flight land before the CTA's shared memory goes
@@ -202,7 +216,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
     }
-    if (POOL) cp_async_wait<0>();
   } else if (warp == 1) {
     // ---------------------------------------------------------------- MMA issuer
     if (lane == 0) {
@@ -348,7 +361,7 @@ csa2_status run_tc(const void* q, const float* w, const void* k, int B, int Q, i
   if (attr_err != cudaSuccess) return fail(CSA2_ERR_CUDA, "index_scores_tc: smem opt-in failed");
   const int64_t grid = std::min<int64_t>(sm_count(), p.n_units);
   begin_launch(stream);
-  kern<<<static_cast<unsigned>(grid), kThreads, C::BYTES, stream>>>(map, p);
+  kern<<<static_cast<unsigned>(grid), POOL ? kPoolThreads : kThreads, C::BYTES, stream>>>(map, p);
   note_launch(POOL ? LK_INDEX_POOL : LK_INDEX, 1, stream);
   return check_launch("index_scores_tc");
 }

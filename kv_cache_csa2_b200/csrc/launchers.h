@@ -16,6 +16,11 @@ csa2_status launch_index_scores(const void* q, const float* w, const void* k, in
                                 int P, csa2_index_act act, float* scores, cudaStream_t stream);
 
 size_t select_topk_workspace(int64_t rows, int64_t L, int count);
+// Two selections of the same rows in one pass set (multi-CTA kernel); returns
+// CSA2_ERR_UNSUPPORTED when that kernel does not apply to the shape.
+csa2_status launch_select_topk2(const float* scores, int64_t rows, int64_t L, int count0,
+                                const int32_t* ids, int32_t* out0, int count1, int32_t* out1,
+                                void* ws, size_t ws_bytes, cudaStream_t stream);
 csa2_status launch_select_topk(const float* scores, int64_t rows, int64_t L, int count,
                                const int32_t* ids, int32_t* out, void* ws, size_t ws_bytes,
                                cudaStream_t stream);
