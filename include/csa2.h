@@ -139,6 +139,26 @@ csa2_status csa2_select_topk(const float* scores, int64_t rows, int64_t L, int c
                              const int32_t* ids, int32_t* out, void* workspace,
                              size_t workspace_bytes, csa2_stream stream);
 
+/* csa2_select_topk without a workspace argument.  The pages have no
+ * counterpart to this call: it is a convenience of this library for callers
+ * that cannot hand out device memory.  Arguments, result and errors are those
+ * of csa2_select_topk (same kernels, bit-identical output); the scratch is a
+ * static device array of CSA2_SELECT_TOPK_NOALLOC_SCRATCH_BYTES per device
+ * inside the library, so the call allocates nothing.
+ *   - A selection that needs more scratch than that (csa2_select_topk_workspace
+ *     of the same arguments) returns CSA2_ERR_OOM with nothing enqueued; at
+ *     L = 262144 the limit is about 40 rows.
+ *   - The part of the scratch that must start at zero is cleared on `stream`
+ *     before every launch (an asynchronous memset, no allocation).
+ *   - The scratch is shared: calls that overlap on one device (other streams,
+ *     other host threads) race on it and give wrong results.  Serialise them.
+ *   - The first call on each device looks up the scratch's address and the
+ *     kernel's occupancy on the host; make one call on a device before
+ *     capturing a stream that contains this call. */
+#define CSA2_SELECT_TOPK_NOALLOC_SCRATCH_BYTES ((size_t)4 << 20)
+csa2_status csa2_select_topk_noalloc(const float* scores, int64_t rows, int64_t L, int count,
+                                     const int32_t* ids, int32_t* out, csa2_stream stream);
+
 /* (a2 + a3) Indexer scores followed by top-k, per layer mode ([V41] CSA2
  * paragraph, hierarchical indexer paragraph; [R] Hierarchical Sparse Indexer):
  *   CSA2_FULL    : pool_in must be NULL.  Scores every visible entry, writes

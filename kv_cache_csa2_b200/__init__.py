@@ -12,7 +12,8 @@ import os
 
 __all__ = [
     "CSA2Error", "lib", "lib_path", "FULL", "REINDEX", "REUSE", "KV_BF16", "KV_FP4", "ACT_RELU",
-    "ACT_IDENTITY", "csa2_compress", "csa2_index_scores", "csa2_select_topk", "csa2_index_topk",
+    "ACT_IDENTITY", "csa2_compress", "csa2_index_scores", "csa2_select_topk", "csa2_select_topk_noalloc",
+    "csa2_index_topk",
     "csa2_sparse_attn", "csa2_fp4_pack", "csa2_fp4_unpack", "Group", "csa2_device_error",
     "launch_counts", "reset_launch_counts", "set_fault", "EXPORTED_SYMBOLS",
 ]
@@ -47,6 +48,7 @@ _SIGS = {
     "csa2_index_scores": (_I, [_P, _P, _P, _I, _I, _I, _I, _I64, _P, _P, _I, _I, _P, _P]),
     "csa2_select_topk_workspace": (_SZ, [_I64, _I64, _I]),
     "csa2_select_topk": (_I, [_P, _I64, _I64, _I, _P, _P, _P, _SZ, _P]),
+    "csa2_select_topk_noalloc": (_I, [_P, _I64, _I64, _I, _P, _P, _P]),
     "csa2_index_topk_workspace": (_SZ, [_I, _I, _I64, _I, _I, _I]),
     "csa2_index_topk": (_I, [_I, _P, _P, _P, _I, _I, _I, _I, _I64, _P, _P, _I, _I, _P, _P, _I, _I,
                              _P, _SZ, _P]),
@@ -188,6 +190,18 @@ def csa2_select_topk(scores, count: int, ids=None, out=None, stream=None):
     ws = _workspace(nb, scores.device)
     _check(lib().csa2_select_topk(_ptr(scores), rows, L, count, _ptr(ids), _ptr(out), _ptr(ws),
                                   nb, _stream(stream)))
+    return out
+
+
+def csa2_select_topk_noalloc(scores, count: int, ids=None, out=None, stream=None):
+    """csa2_select_topk with the library's static scratch (no workspace is allocated)."""
+    torch = _torch()
+    L = scores.shape[-1]
+    rows = scores.numel() // max(L, 1)
+    if out is None:
+        out = torch.empty(*scores.shape[:-1], count, dtype=torch.int32, device=scores.device)
+    _check(lib().csa2_select_topk_noalloc(_ptr(scores), rows, L, count, _ptr(ids), _ptr(out),
+                                          _stream(stream)))
     return out
 
 
