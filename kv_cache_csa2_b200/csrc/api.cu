@@ -162,6 +162,32 @@ static size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
   } while (0)
 #define REQUIRE_PTR(p) REQUIRE((p) != nullptr && aligned16(p), "%s: pointer " #p " is null or not 16-byte aligned", __func__)
 
+namespace csa2 {
+csa2_status sparse_attn_checked(csa2_mode mode, const void* q, const csa2_kv* kv,
+                                const int32_t* topk, int B, int Q, int Ha, int k, float scale,
+                                void* out, float* lse, void* workspace, size_t workspace_bytes,
+                                unsigned long long* sync_zeroed, cudaStream_t stream) {
+  CSA2_TRY(fault_gate());
+  REQUIRE(mode == CSA2_FULL || mode == CSA2_REINDEX || mode == CSA2_REUSE,
+          "csa2_sparse_attn: unknown mode %d", int(mode));
+  REQUIRE(kv != nullptr, "csa2_sparse_attn: kv is null");
+  REQUIRE(B >= 0 && Q >= 0 && k >= 0 && Ha > 0, "csa2_sparse_attn: bad size");
+  REQUIRE(kv->fmt == CSA2_KV_BF16 || kv->fmt == CSA2_KV_FP4, "csa2_sparse_attn: unknown kv format");
+  REQUIRE(kv->dim > 0 && kv->dim % 16 == 0, "csa2_sparse_attn: D=%d must be a multiple of 16", kv->dim);
+  REQUIRE(kv->n >= 0 && kv->n <= 0x7fffffffLL, "csa2_sparse_attn: bad kv->n");
+  if (B == 0 || Q == 0) return CSA2_OK;
+  REQUIRE_PTR(q); REQUIRE_PTR(out); REQUIRE_PTR(kv->data);
+  REQUIRE(k == 0 || topk != nullptr, "csa2_sparse_attn: topk is null");
+  REQUIRE(kv->fmt == CSA2_KV_BF16 || kv->scales != nullptr, "csa2_sparse_attn: FP4 kv without scales");
+  const size_t need = sparse_attn_workspace(B, Q, Ha, kv->dim, k, kv->fmt);
+  if (workspace_bytes < need || (need > 0 && !workspace))
+    return fail(CSA2_ERR_OOM, "csa2_sparse_attn: workspace %zu < %zu bytes", workspace_bytes, need);
+  return launch_sparse_attn(q, *kv, topk, B, Q, Ha, k, scale, out, lse, workspace, workspace_bytes,
+                            sync_zeroed, stream);
+}
+}  // namespace csa2
+
+
 extern "C" {
 
 const char* csa2_status_string(csa2_status s) {
@@ -387,23 +413,8 @@ csa2_status csa2_sparse_attn(csa2_mode mode, const void* q, const csa2_kv* kv,
                              const int32_t* topk, int B, int Q, int Ha, int k, float scale,
                              void* out, float* lse, void* workspace, size_t workspace_bytes,
                              csa2_stream stream) {
-  CSA2_TRY(fault_gate());
-  REQUIRE(mode == CSA2_FULL || mode == CSA2_REINDEX || mode == CSA2_REUSE,
-          "csa2_sparse_attn: unknown mode %d", int(mode));
-  REQUIRE(kv != nullptr, "csa2_sparse_attn: kv is null");
-  REQUIRE(B >= 0 && Q >= 0 && k >= 0 && Ha > 0, "csa2_sparse_attn: bad size");
-  REQUIRE(kv->fmt == CSA2_KV_BF16 || kv->fmt == CSA2_KV_FP4, "csa2_sparse_attn: unknown kv format");
-  REQUIRE(kv->dim > 0 && kv->dim % 16 == 0, "csa2_sparse_attn: D=%d must be a multiple of 16", kv->dim);
-  REQUIRE(kv->n >= 0 && kv->n <= 0x7fffffffLL, "csa2_sparse_attn: bad kv->n");
-  if (B == 0 || Q == 0) return CSA2_OK;
-  REQUIRE_PTR(q); REQUIRE_PTR(out); REQUIRE_PTR(kv->data);
-  REQUIRE(k == 0 || topk != nullptr, "csa2_sparse_attn: topk is null");
-  REQUIRE(kv->fmt == CSA2_KV_BF16 || kv->scales != nullptr, "csa2_sparse_attn: FP4 kv without scales");
-  const size_t need = sparse_attn_workspace(B, Q, Ha, kv->dim, k, kv->fmt);
-  if (workspace_bytes < need || (need > 0 && !workspace))
-    return fail(CSA2_ERR_OOM, "csa2_sparse_attn: workspace %zu < %zu bytes", workspace_bytes, need);
-  return launch_sparse_attn(q, *kv, topk, B, Q, Ha, k, scale, out, lse, workspace, workspace_bytes,
-                            reinterpret_cast<cudaStream_t>(stream));
+  return sparse_attn_checked(mode, q, kv, topk, B, Q, Ha, k, scale, out, lse, workspace,
+                             workspace_bytes, nullptr, reinterpret_cast<cudaStream_t>(stream));
 }
 
 // ------------------------------------------------------------- (a5)

@@ -17,7 +17,8 @@ namespace csa2 {
 
 csa2_status launch_sparse_attn_tc(const void* q, const csa2_kv& kv, const int32_t* topk, int B,
                                   int Q, int Ha, int k, float scale, void* out, float* lse,
-                                  void* ws, size_t ws_bytes, cudaStream_t stream);
+                                  void* ws, size_t ws_bytes, unsigned long long* sync_zeroed,
+                                  cudaStream_t stream);
 size_t sparse_attn_tc_workspace(int B, int Q, int Ha, int D, int k, csa2_kv_fmt fmt);
 
 namespace {
@@ -206,10 +207,11 @@ size_t sparse_attn_workspace(int B, int Q, int Ha, int D, int k, csa2_kv_fmt fmt
 
 csa2_status launch_sparse_attn(const void* q, const csa2_kv& kv, const int32_t* topk, int B,
                                int Q, int Ha, int k, float scale, void* out, float* lse, void* ws,
-                               size_t ws_bytes, cudaStream_t stream) {
+                               size_t ws_bytes, unsigned long long* sync_zeroed,
+                               cudaStream_t stream) {
   if (B == 0 || Q == 0) return CSA2_OK;
   csa2_status s = launch_sparse_attn_tc(q, kv, topk, B, Q, Ha, k, scale, out, lse, ws, ws_bytes,
-                                        stream);
+                                        sync_zeroed, stream);
   if (s != CSA2_ERR_UNSUPPORTED) return s;
   const int D = kv.dim;
   if (Ha == 64 && D == 512) return run_simt<64, 512>(q, kv, topk, B, Q, k, scale, out, lse, stream);

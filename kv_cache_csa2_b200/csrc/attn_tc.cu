@@ -5,32 +5,32 @@
 // reduction order is fixed and does not depend on the batch.
 //
 // Shapes: 64 heads, entries of width 512, bf16.  A query's k selected rows are
-// cut into tiles of 128 rows, one tile per CTA; the tiles of a query are
-// spread over NCL thread-block clusters of CS CTAs (CS = 4, or 2 when k
-// fits two tiles; NCL = tiles/CS <= 16; both fixed by k alone).  Per CTA:
-//   warp 0     loads the query's 64 x 512 heads (TMA) and gathers the tile's
-//              128 selected rows with TMA row gathers (4 rows x 128 bytes per
-//              instruction, issued by all 32 lanes, one barrier per 64-column
-//              block so the first MMAs start early) into a 128-byte-swizzled
-//              tile; empty slots gather a real row and are masked out;
-//   warp 1     allocates TMEM and issues the MMAs:
-//                S^T[row, head] = KV[row, :] . q[head, :]    (M=128, N=64, K=512)
-//                O^T[dim, head] += KV[row, dim] * P[row, head] (M=128 dims x4, N=64, K=128)
-//              both products read the same tile through K-major and MN-major
-//              descriptors (no transposes);
-//   warps 2-5  softmax with the tile's own per-head max m (P in bf16 for the
-//              PV product, row sums l in f32), then the reductions.
-// Cluster reduction: every CTA pushes (m, l) to its peers over distributed
-// shared memory and stages its partial O^T in its own shared memory; after a
-// cluster barrier the CTA that owns dims [r*512/CS, (r+1)*512/CS) reads that
-// slice from every peer and adds them in rank order, each weighted by
-// exp(m_c - M) with M the cluster's max.  With one cluster per query the owner
-// divides by L and writes out (bf16) and lse.  With several, each owner writes
-// its (O, M, L) slice to a global workspace and takes a ticket; the owner that
-// arrives last merges the NCL slices in cluster order (same weighting) and
-// writes out -- no CTA waits for another cluster.  Three cluster barriers;
-// every other wait is bounded (2 s), and a CTA that gives up still takes part
-// in every cluster barrier.
+// cut into T = ceil(k / 128) tiles of 128 rows and each (query, tile) unit runs
+// on one CTA.  The CTA computes its tile's partial result with the tile's own
+// per-head max m (P = exp(s - m) rounded to bf16, l = sum of P, O = P^T KV in
+// f32), writes (O, m, l) to a global workspace and meets the query's other
+// T - 1 CTAs at a counter in global memory.  CTA t then reduces output dims
+// [t * dpc, (t + 1) * dpc) over the T partials in tile order, each weighted by
+// exp(m_j - M) with M = max_j m_j, divides by L = sum_j l_j exp(m_j - M) and
+// writes bf16 out (tile 0 also lse = M + log L).  The launch is cooperative:
+// the whole grid is resident, so the counter wait always ends.  A grid holds
+// the units of G queries and loops over the batch in waves of G queries.  The
+// split and the reduction order depend on k only, so results are
+// deterministic and batch-invariant.
+//
+// Per CTA (6 warps):
+//   warp 0     TMA load of the query's 64 x 512 heads, once per wave;
+//   warp 1     TMEM allocation and MMA issue:
+//                S^T[row, head]  = KV[row, :] . q[head, :]      (M=128, N=64, K=512)
+//                O^T[dim, head] += KV[row, dim] * P[row, head]  (M=128 x4, N=64, K=128)
+//              both read the same tile through K-major and MN-major descriptors;
+//   warps 2-5  gather of the tile's 128 rows (16-byte cp.async copies straight
+//              into the 128-byte-swizzled layout, 64 per thread in flight; the
+//              next wave's gather is issued as soon as this wave's products are
+//              done), softmax, partial write, counter wait, reduction, output.
+// Every wait is bounded (mbarriers 2 s, the counter 1 s); a CTA that gives up
+// records CSA2_ERR_TIMEOUT and still takes every later step, so no other CTA
+// waits for it in vain.
 #include <algorithm>
 #include <cstdlib>
 #include <cstring>
@@ -50,36 +50,40 @@ constexpr int kRows = 128;                    // rows per tile (MMA M of S^T)
 constexpr int kThreads = 6 * 32;
 constexpr int kKB = DV / 64;                  // 8 K-blocks of 64 dims
 constexpr int kKBBytes = kRows * 128;         // 16 KiB
-constexpr int kMinCS = 2;                     // an owner's slice must fit the q region
-constexpr int kMaxCS = 8;
-constexpr int kDefaultCS = 4;
-constexpr int kMaxNCL = 2 * kMaxCS;           // clusters per query: weights live in the (m, l) region
-constexpr int kStageStride = HA + 4;          // floats per staged dim row: 272 B
+constexpr int kMaxTiles = 64;                 // k <= 8192
+constexpr int kPartFloats = DV * HA;          // partial O^T [dim][head], 128 KiB
+constexpr int kSlotFloats = kPartFloats + 2 * HA;   // + the tile's m[HA], l[HA]
 
 constexpr int OFF_KV = 0;                              // 128 KiB: KV tile
 constexpr int OFF_P = OFF_KV + kKB * kKBBytes;         // 16 KiB: P tile
-constexpr int OFF_Q = OFF_P + kRows * 128;             // 64 KiB: q (8 K-blocks x 64 rows)
-constexpr int OFF_ML = OFF_Q + kKB * HA * 128;         // [kMaxCS][2][HA] f32 (m, l), written by peers
-constexpr int OFF_RED = OFF_ML + kMaxCS * 2 * HA * 4;  // [4 warps][HA] f32
-constexpr int OFF_W = OFF_RED + 4 * HA * 4;            // [kMaxCS][HA] f32 weights, [HA] M, [HA] L
-constexpr int OFF_BAR = OFF_W + (kMaxCS + 2) * HA * 4;
+constexpr int OFF_Q = OFF_P + kRows * 128;             // 64 KiB: q; after the products, the reduction's scratch
+constexpr int OFF_RED = OFF_Q + kKB * HA * 128;        // [4 warps][HA] f32
+constexpr int OFF_ML = OFF_RED + 4 * HA * 4;           // this tile's m[HA], l[HA]
+constexpr int OFF_ML2 = OFF_ML + 2 * HA * 4;           // the query's M[HA], L[HA]
+constexpr int OFF_BAR = OFF_ML2 + 2 * HA * 4;
 constexpr int NBAR = 16;
 constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
 constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;
-static_assert(DV * kStageStride * 4 <= OFF_Q, "partial O^T staged in the KV + P region");
-static_assert(HA * (DV / kMinCS) * 4 <= kKB * HA * 128, "an owner's slice fits the q region");
+// reduction scratch inside the q region: output staging [HA][kStageStride]
+// f32 for up to kStageDims dims, then per-tile weights and row sums [T][HA] f32
+constexpr int kStageDims = 64;
+constexpr int kStageStride = kStageDims + 1;
+constexpr int kWeightsOff = HA * kStageStride * 4;
+static_assert(kWeightsOff % 16 == 0 && kWeightsOff + 2 * kMaxTiles * HA * 4 <= kKB * HA * 128,
+              "staging, weights and row sums fit the q region");
 static_assert(SMEM_BYTES <= 232448, "shared memory");
-static_assert(kMaxNCL * HA <= kMaxCS * 2 * HA, "per-cluster weights fit the (m, l) region");
 
 struct Params {
-  const int32_t* topk;     // [B*Q, k]
-  uint16_t* out;           // [B*Q, 64, 512]
-  float* lse;              // [B*Q, 64] or null
-  float* part;             // [B*Q][ncl][cs][dpo*64 + 2*64] cross-cluster slices (ncl > 1)
-  unsigned* ticket;        // [B*Q][cs], zero before the launch (ncl > 1)
+  const int32_t* topk;             // [B*Q, k]
+  const uint16_t* kv;              // [B, n, 512]
+  uint16_t* out;                   // [B*Q, 64, 512]
+  float* lse;                      // [B*Q, 64] or null
+  float* part;                     // [2][grid][kSlotFloats]
+  unsigned long long* sync;        // [G] arrival counters (multiples of T between launches)
   int* err;
-  int64_t n;
-  int Q, k, cs, ncl;
+  int64_t n, n_queries;
+  int Q, k, T, G, dpc;
+  int bulk;                        // a CTA's dims of all T partials fit the KV region, their (m, l) the P region
   float scale;
 };
 
@@ -114,52 +118,60 @@ __device__ __forceinline__ float rescale(float m, float M) {
   return (m == -INFINITY || M == -INFINITY) ? 0.0f : __expf(m - M);
 }
 
+__device__ __forceinline__ unsigned long long ld_acquire_u64(const unsigned long long* p) {
+  unsigned long long v;
+  asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+  return v;
+}
+
+// Drops a 128-byte line from L2 without writing it back (its content becomes
+// undefined); used on workspace lines that no one reads again.
+__device__ __forceinline__ void discard_l2_line(const void* p) {
+  asm volatile("discard.global.L2 [%0], 128;" ::"l"(p) : "memory");
+}
+
 __global__ void __launch_bounds__(kThreads, 1)
-    attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap kvmap,
-                   const Params p) {
+    attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const Params p) {
   extern __shared__ uint8_t smem_raw[];
-  __shared__ unsigned sh_ticket;
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sKV = smem + OFF_KV;
   uint8_t* sP = smem + OFF_P;
   uint8_t* sQ = smem + OFF_Q;
-  float* sML = reinterpret_cast<float*>(smem + OFF_ML);     // [c][0][h] = m_c, [c][1][h] = l_c
   float* sRed = reinterpret_cast<float*>(smem + OFF_RED);
-  float* sWt = reinterpret_cast<float*>(smem + OFF_W);      // [c][h] weights exp(m_c - M)
-  float* sMcl = sWt + kMaxCS * HA;                          // [h] max M
-  float* sLcl = sMcl + HA;                                  // [h] sum L
-  float* sStage = reinterpret_cast<float*>(smem + OFF_KV);
+  float* sML = reinterpret_cast<float*>(smem + OFF_ML);      // m[HA], l[HA] of this tile
+  float* sML2 = reinterpret_cast<float*>(smem + OFF_ML2);    // M[HA], L[HA] of the query
+  float* sStage = reinterpret_cast<float*>(sQ);              // [HA][kStageStride]
+  float* sW = reinterpret_cast<float*>(sQ + kWeightsOff);    // [T][HA] weights
+  float* sLv = sW + kMaxTiles * HA;                          // [T][HA] row sums l_j
   uint64_t* bar = reinterpret_cast<uint64_t*>(smem + OFF_BAR);
   uint64_t* q_full = bar + 0;
-  uint64_t* p_full = bar + 1;
-  uint64_t* o_full = bar + 2;
-  uint64_t* s_full = bar + 3;
+  uint64_t* s_full = bar + 1;
+  uint64_t* p_full = bar + 2;
+  uint64_t* o_full = bar + 3;
+  uint64_t* m_done = bar + 4;                  // the reduction no longer needs the q region
+  uint64_t* r_full = bar + 5;                  // this CTA's dims of every partial are in the KV region
   uint64_t* kv_full = bar + 8;                 // [8]: one per 64-column block of the tile
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + OFF_MISC + 4);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int cs = p.cs;
-  const uint32_t me = cluster_rank();
-  const int64_t per_query = static_cast<int64_t>(cs) * p.ncl;
-  const int64_t qi = blockIdx.x / per_query;                      // flat (b, q)
-  const int cl = static_cast<int>((blockIdx.x % per_query) / cs); // cluster index within the query
-  const int tile = cl * cs + static_cast<int>(me);
-  const int64_t b = qi / p.Q;
-  const int32_t* ids = p.topk + qi * p.k;
+  const int tile = static_cast<int>(blockIdx.x % p.T);
+  const int slot = static_cast<int>(blockIdx.x / p.T);        // query slot: queries slot, slot+G, ...
+  const int64_t n_waves = (p.n_queries - slot + p.G - 1) / p.G;
   constexpr uint32_t S_COL = 0;                       // S at columns [0, 64)
   constexpr uint32_t O_COL = 256;                     // O^T chunk mc at [256 + 64 mc, ...)
 
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
+    mbar_init(s_full, 1);
     mbar_init(p_full, 4);
     mbar_init(o_full, 1);
-    mbar_init(s_full, 1);
-    for (int kb = 0; kb < kKB; ++kb) mbar_init(&kv_full[kb], 1);
+    mbar_init(m_done, 1);
+    mbar_init(r_full, 1);
+    for (int kb = 0; kb < kKB; ++kb) mbar_init(&kv_full[kb], 128);
     *abort_flag = 0;
     fence_mbar_init();
     prefetch_tensor_map(&qmap);
-    prefetch_tensor_map(&kvmap);
   }
   if (warp == 1) {
     tmem_alloc(tmem_slot, 512);
@@ -169,59 +181,51 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  cluster_sync_all();          // barrier 0: every CTA of the cluster is running before peers write to it
 
   if (warp == 0) {
-    // ------------------------------------------------------------ producer
+    // ------------------------------------------------------------ q loader
     if (lane == 0) {
-      mbar_arrive_expect_tx(q_full, HA * DV * 2);
+      int64_t issued = 0;
+      for (int64_t w = 0; w < n_waves; ++w) {
+        if (w > 0 && !mbar_wait(m_done, static_cast<uint32_t>((w - 1) & 1), abort_flag, p.err)) break;
+        const int64_t qi = slot + w * p.G;
+        mbar_arrive_expect_tx(q_full, HA * DV * 2);
 #pragma unroll
-      for (int kb = 0; kb < kKB; ++kb)
-        tma_load_2d(sQ + kb * HA * 128, &qmap, q_full, kb * 64, static_cast<int32_t>(qi * HA));
-    }
-    // lane g gathers rows 4g .. 4g+3 of the tile, one 64-column block at a time
-    const int32_t seq_row0 = static_cast<int32_t>(b * p.n);
-    const int64_t pos0 = static_cast<int64_t>(tile) * kRows + 4 * lane;
-    int32_t row[4];
-#pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      int id = pos0 + u < p.k ? ids[pos0 + u] : -1;
-      if (id >= p.n || id < -1) {
-        raise_dev_error(p.err, DEVERR_BOUNDS);
-        id = -1;
+        for (int kb = 0; kb < kKB; ++kb)
+          tma_load_2d(sQ + kb * HA * 128, &qmap, q_full, kb * 64, static_cast<int32_t>(qi * HA));
+        issued = w + 1;
       }
-      row[u] = seq_row0 + (id >= 0 ? id : 0);          // empty slot: masked later
-    }
-#pragma unroll
-    for (int kb = 0; kb < kKB; ++kb) {
-      if (lane == 0) mbar_arrive_expect_tx(&kv_full[kb], kRows * 128);
-      __syncwarp();
-      tma_gather4(sKV + kb * kKBBytes + 4 * lane * 128, &kvmap, &kv_full[kb], kb * 64, row[0], row[1],
-                  row[2], row[3]);
+      // the last load has landed before the CTA may exit (bounded: 0.1 s)
+      if (issued > 0) {
+        const uint64_t t0 = globaltimer_ns();
+        while (!mbar_try_wait(q_full, static_cast<uint32_t>((issued - 1) & 1)) &&
+               globaltimer_ns() - t0 < 100000000ull) {
+        }
+      }
     }
     __syncwarp();
-    cluster_sync_all();                                // barrier 1
-    cluster_sync_all();                                // barrier 2
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     constexpr uint32_t idesc_s = idesc_bf16_f32(128, HA, false, false);
     constexpr uint32_t idesc_o = idesc_bf16_f32(128, HA, true, true);
     const uint32_t kv0 = smem_u32(sKV), q0 = smem_u32(sQ), p0 = smem_u32(sP);
     if (lane == 0) {
-      bool ok = mbar_wait(q_full, 0, abort_flag, p.err);
+      for (int64_t w = 0; w < n_waves; ++w) {
+        const uint32_t par = static_cast<uint32_t>(w & 1);
+        bool ok = mbar_wait(q_full, par, abort_flag, p.err);
 #pragma unroll 1
-      for (int kb = 0; kb < kKB && ok; ++kb) {
-        ok = mbar_wait(&kv_full[kb], 0, abort_flag, p.err);
-        if (!ok) break;
-        tc_fence_after();
+        for (int kb = 0; kb < kKB && ok; ++kb) {
+          ok = mbar_wait(&kv_full[kb], par, abort_flag, p.err);
+          if (!ok) break;
+          tc_fence_after();
 #pragma unroll
-        for (int kk = 0; kk < 4; ++kk)
-          mma_bf16(tmem + S_COL, desc_kmajor_sw128(kv0 + kb * kKBBytes + kk * 32),
-                   desc_kmajor_sw128(q0 + kb * HA * 128 + kk * 32), idesc_s, (kb | kk) != 0);
-      }
-      if (ok) mma_commit(s_full);
-      if (ok) ok = mbar_wait(p_full, 0, abort_flag, p.err);
-      if (ok) {
+          for (int kk = 0; kk < 4; ++kk)
+            mma_bf16(tmem + S_COL, desc_kmajor_sw128(kv0 + kb * kKBBytes + kk * 32),
+                     desc_kmajor_sw128(q0 + kb * HA * 128 + kk * 32), idesc_s, (kb | kk) != 0);
+        }
+        if (!ok) break;
+        mma_commit(s_full);
+        if (!mbar_wait(p_full, par, abort_flag, p.err)) break;
         tc_fence_after();
 #pragma unroll
         for (int mc = 0; mc < 4; ++mc)
@@ -234,248 +238,335 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
     __syncwarp();
-    cluster_sync_all();                                // barrier 1
-    cluster_sync_all();                                // barrier 2
   } else {
-    // ------------------------------------------------------------ softmax + reductions
+    // ------------------------------------------------------------ gather, softmax, reduction
     const int quad = warp & 3;
     const int ew = warp - 2;                           // epilogue warp 0..3
     const int row = quad * 32 + lane;                  // TMEM lane = tile row
     const int et = ew * 32 + lane;                     // epilogue thread 0..127
     const uint32_t lane_off = static_cast<uint32_t>(quad * 32) << 16;
-    const int64_t pos = static_cast<int64_t>(tile) * kRows + row;
-    const int64_t id = pos < p.k ? ids[pos] : -1;
-    const bool valid = id >= 0 && id < p.n;
     const int hb = reduced_head_base(lane);
-    bool ok = mbar_wait(s_full, 0, abort_flag, p.err);
-    float x[HA];
-    if (ok) {
-      tc_fence_after();
-      uint32_t v[32];
+    // gather: thread et copies 16-byte chunk c16 of rows grow0 + 16 i (i < 8)
+    // in every 64-column block; eight consecutive threads cover one 128-byte
+    // row segment.  (grow0 + 16 i) & 7 == grow0 & 7: one swizzle per thread.
+    const int c16 = et & 7, grow0 = et >> 3;
+    const uint32_t swz = static_cast<uint32_t>((c16 ^ (grow0 & 7)) << 4);
+    auto issue_gather = [&](int64_t qi) {
+      const uint16_t* base = p.kv + (qi / p.Q) * p.n * DV + c16 * 8;
+      const int32_t* ids = p.topk + qi * p.k;
+      int64_t off[8];
 #pragma unroll
-      for (int half = 0; half < 2; ++half) {
-        tmem_ld32(tmem + lane_off + S_COL + 32 * half, v);
-        tmem_wait_ld();
-#pragma unroll
-        for (int h = 0; h < 32; ++h) x[32 * half + h] = valid ? p.scale * __uint_as_float(v[h]) : -INFINITY;
-      }
-    } else {
-#pragma unroll
-      for (int h = 0; h < HA; ++h) x[h] = -INFINITY;
-    }
-    // the tile's per-head max m
-    float red[HA];
-#pragma unroll
-    for (int h = 0; h < HA; ++h) red[h] = x[h];
-    warp_transpose_reduce<true>(red, lane);
-    sRed[ew * HA + hb] = red[0];
-    sRed[ew * HA + hb + 1] = red[1];
-    epi_bar();
-    float* mine = sML + me * 2 * HA;                   // this CTA's (m, l) slot (also in every peer)
-    if (et < HA)
-      mine[et] = fmaxf(fmaxf(sRed[et], sRed[HA + et]), fmaxf(sRed[2 * HA + et], sRed[3 * HA + et]));
-    epi_bar();
-    // P = exp(x - m) in bf16, and its row sums
-    float lsum[HA];
-    {
-      uint32_t packed[32];
-#pragma unroll
-      for (int h2 = 0; h2 < 32; ++h2) {
-        float e[2];
-#pragma unroll
-        for (int u = 0; u < 2; ++u) {
-          const int h = 2 * h2 + u;
-          e[u] = (x[h] == -INFINITY) ? 0.0f : __expf(x[h] - mine[h]);
+      for (int i = 0; i < 8; ++i) {
+        const int64_t pos = static_cast<int64_t>(tile) * kRows + grow0 + 16 * i;
+        int id = pos < p.k ? ids[pos] : -1;
+        if (id >= p.n || id < -1) {
+          raise_dev_error(p.err, DEVERR_BOUNDS);
+          id = -1;
         }
-        packed[h2] = pack_bf16x2(e[0], e[1]);
-        lsum[2 * h2] = bf16_lo(packed[h2]);
-        lsum[2 * h2 + 1] = bf16_hi(packed[h2]);
+        off[i] = static_cast<int64_t>(id >= 0 ? id : 0) * DV;     // empty slot: masked later
       }
 #pragma unroll
-      for (int c = 0; c < 8; ++c)
-        *reinterpret_cast<uint4*>(sP + sw128_offset(row, c)) =
-            make_uint4(packed[4 * c], packed[4 * c + 1], packed[4 * c + 2], packed[4 * c + 3]);
+      for (int kb = 0; kb < kKB; ++kb) {
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+          cp_async_16(sKV + kb * kKBBytes + (grow0 + 16 * i) * 128 + swz, base + off[i] + kb * 64, 16);
+        cp_async_commit();
+      }
+    };
+    // each 64-column block is published once this thread's copies into it landed
+    auto publish_gather = [&]() {
+#define CSA2_PUBLISH(KB)            \
+  cp_async_wait<kKB - 1 - (KB)>();  \
+  fence_proxy_async_smem();         \
+  mbar_arrive(&kv_full[KB]);
+      CSA2_PUBLISH(0) CSA2_PUBLISH(1) CSA2_PUBLISH(2) CSA2_PUBLISH(3)
+      CSA2_PUBLISH(4) CSA2_PUBLISH(5) CSA2_PUBLISH(6) CSA2_PUBLISH(7)
+#undef CSA2_PUBLISH
+    };
+    if (n_waves > 0) {
+      issue_gather(slot);
+      publish_gather();
     }
-    fence_proxy_async_smem();
-    __syncwarp();
-    if (lane == 0) mbar_arrive(p_full);
-    warp_transpose_reduce<false>(lsum, lane);
-    sRed[ew * HA + hb] = lsum[0];
-    sRed[ew * HA + hb + 1] = lsum[1];
-    epi_bar();
-    if (et < HA) mine[HA + et] = (sRed[et] + sRed[HA + et]) + (sRed[2 * HA + et] + sRed[3 * HA + et]);
-    epi_bar();
-    // push (m, l) to every peer
-    for (int i = et; i < cs * 2 * HA; i += 128) {
-      const int dst = i / (2 * HA), j = i % (2 * HA);
-      if (dst != static_cast<int>(me)) st_cluster_f32(map_to_rank(smem_u32(&mine[j]), dst), mine[j]);
-    }
-    // stage the partial O^T [dim][head] in this CTA's own KV + P region
-    if (ok) ok = mbar_wait(o_full, 0, abort_flag, p.err);
-    if (ok) {
-      tc_fence_after();
-#pragma unroll 1
-      for (int mc = 0; mc < 4; ++mc) {
-        float* dst = sStage + (mc * 128 + row) * kStageStride;
+    bool ok = true;
+    for (int64_t w = 0; w < n_waves; ++w) {
+      const int64_t qi = slot + w * p.G;
+      const uint32_t par = static_cast<uint32_t>(w & 1);
+      const int64_t pos = static_cast<int64_t>(tile) * kRows + row;
+      const int64_t id = pos < p.k ? p.topk[qi * p.k + pos] : -1;
+      const bool valid = id >= 0 && id < p.n;
+      ok = ok && mbar_wait(s_full, par, abort_flag, p.err);
+      float x[HA];
+      if (ok) {
+        tc_fence_after();
+        uint32_t v[32];
 #pragma unroll
         for (int half = 0; half < 2; ++half) {
-          uint32_t v[32];
-          tmem_ld32(tmem + lane_off + O_COL + 64 * mc + 32 * half, v);
+          tmem_ld32(tmem + lane_off + S_COL + 32 * half, v);
           tmem_wait_ld();
 #pragma unroll
-          for (int c = 0; c < 8; ++c)
-            *reinterpret_cast<float4*>(dst + 32 * half + 4 * c) =
-                make_float4(__uint_as_float(v[4 * c]), __uint_as_float(v[4 * c + 1]),
-                            __uint_as_float(v[4 * c + 2]), __uint_as_float(v[4 * c + 3]));
+          for (int h = 0; h < 32; ++h) x[32 * half + h] = valid ? p.scale * __uint_as_float(v[h]) : -INFINITY;
+        }
+      } else {
+#pragma unroll
+        for (int h = 0; h < HA; ++h) x[h] = -INFINITY;
+      }
+      // the tile's per-head max m
+      {
+        float red[HA];
+#pragma unroll
+        for (int h = 0; h < HA; ++h) red[h] = x[h];
+        warp_transpose_reduce<true>(red, lane);
+        sRed[ew * HA + hb] = red[0];
+        sRed[ew * HA + hb + 1] = red[1];
+      }
+      epi_bar();
+      if (et < HA)
+        sML[et] = fmaxf(fmaxf(sRed[et], sRed[HA + et]), fmaxf(sRed[2 * HA + et], sRed[3 * HA + et]));
+      epi_bar();
+      // P = exp(x - m) in bf16, and its row sums
+      float lsum[HA];
+      {
+        const uint32_t ml0 = smem_u32(sML), p0 = smem_u32(sP);
+        uint32_t packed[32];
+#pragma unroll
+        for (int h4 = 0; h4 < HA / 4; ++h4) {
+          const float4 m4 = lds_v4f(ml0 + 16 * h4);
+          const float mm[4] = {m4.x, m4.y, m4.z, m4.w};
+#pragma unroll
+          for (int u = 0; u < 2; ++u) {
+            const int h = 4 * h4 + 2 * u;
+            const float e0 = (x[h] == -INFINITY) ? 0.0f : __expf(x[h] - mm[2 * u]);
+            const float e1 = (x[h + 1] == -INFINITY) ? 0.0f : __expf(x[h + 1] - mm[2 * u + 1]);
+            const uint32_t pk = pack_bf16x2(e0, e1);
+            packed[2 * h4 + u] = pk;
+            lsum[h] = bf16_lo(pk);
+            lsum[h + 1] = bf16_hi(pk);
+          }
+        }
+#pragma unroll
+        for (int c = 0; c < 8; ++c)
+          sts_v4u(p0 + sw128_offset(row, c), packed[4 * c], packed[4 * c + 1], packed[4 * c + 2], packed[4 * c + 3]);
+      }
+      fence_proxy_async_smem();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(p_full);
+      warp_transpose_reduce<false>(lsum, lane);
+      sRed[ew * HA + hb] = lsum[0];
+      sRed[ew * HA + hb + 1] = lsum[1];
+      epi_bar();
+      if (et < HA) sML[HA + et] = (sRed[et] + sRed[HA + et]) + (sRed[2 * HA + et] + sRed[3 * HA + et]);
+      // partial (O^T, m, l) of this tile to workspace slot (buffer w & 1, CTA).
+      // O^T is staged in the KV region as [dim][16 chunks of 4 heads] with
+      // chunk h4 at position h4 ^ (dim & 7) (conflict-free) and written with
+      // (m, l) by two bulk stores; the slot keeps that layout.
+      ok = ok && mbar_wait(o_full, par, abort_flag, p.err);
+      tc_fence_after();
+      const bool more = w + 1 < n_waves;
+      const int64_t buf = (w & 1) * static_cast<int64_t>(gridDim.x);
+      const uint32_t kv0 = smem_u32(sKV);
+      float* my_slot = p.part + (buf + blockIdx.x) * kSlotFloats;
+#pragma unroll 1
+      for (int mc = 0; mc < 4; ++mc) {
+        const int dim = mc * 128 + row;
+        const uint32_t srow = kv0 + dim * (HA * 4);
+        if (ok) {
+#pragma unroll
+          for (int half = 0; half < 2; ++half) {
+            uint32_t v[32];
+            tmem_ld32(tmem + lane_off + O_COL + 64 * mc + 32 * half, v);
+            tmem_wait_ld();
+#pragma unroll
+            for (int c = 0; c < 8; ++c)
+              sts_v4u(srow + (((8 * half + c) ^ (dim & 7)) << 4), v[4 * c], v[4 * c + 1], v[4 * c + 2], v[4 * c + 3]);
+          }
+        }
+        fence_proxy_async_smem();
+        epi_bar();                                     // chunk mc staged (and, at mc = 3, l is in sML)
+        if (et == 0) {
+          bulk_store(my_slot + mc * 128 * HA, sKV + mc * 128 * HA * 4, 128 * HA * 4);
+          if (mc == 3) bulk_store(my_slot + kPartFloats, sML, 2 * HA * 4);
+          bulk_commit();
         }
       }
-    }
-    tc_fence_before();
-    __syncwarp();
-    cluster_sync_all();                                // barrier 1: every partial and (m, l) is in place
-    // cluster max M, per-peer weights, cluster sum L
-    if (et < HA) {
-      float M = -INFINITY;
-      for (int c = 0; c < cs; ++c) M = fmaxf(M, sML[c * 2 * HA + et]);
-      float L = 0.0f;
-      for (int c = 0; c < cs; ++c) {
-        const float wgt = rescale(sML[c * 2 * HA + et], M);
-        sWt[c * HA + et] = wgt;
-        L += sML[c * 2 * HA + HA + et] * wgt;
-      }
-      sMcl[et] = M;
-      sLcl[et] = L;
-    }
-    epi_bar();
-    // pull this CTA's dims from every peer (16-byte chunks, consecutive threads
-    // read consecutive chunks of a staged row) and add them in rank order
-    const int dpo = DV / cs;                           // dims per owner
-    float* sOwn = reinterpret_cast<float*>(sQ);        // [HA][dpo] f32 (q is no longer needed)
-    const uint32_t stage0 = smem_u32(sStage);
-#pragma unroll 2
-    for (int ci = et; ci < dpo * (HA / 4); ci += 128) {
-      const int dl = ci / (HA / 4), h4 = ci % (HA / 4);
-      const uint32_t off = ((static_cast<uint32_t>(me) * dpo + dl) * kStageStride + 4 * h4) * 4;
-      float4 part[kMaxCS];
-#pragma unroll
-      for (int c = 0; c < kMaxCS; ++c)
-        if (c < cs) part[c] = ld_cluster_v4(map_to_rank(stage0 + off, c));
-      float a[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-      for (int c = 0; c < kMaxCS; ++c) {
-        if (c < cs) {
-          a[0] += part[c].x * sWt[c * HA + 4 * h4];
-          a[1] += part[c].y * sWt[c * HA + 4 * h4 + 1];
-          a[2] += part[c].z * sWt[c * HA + 4 * h4 + 2];
-          a[3] += part[c].w * sWt[c * HA + 4 * h4 + 3];
-        }
-      }
-#pragma unroll
-      for (int u = 0; u < 4; ++u) sOwn[(4 * h4 + u) * dpo + dl] = a[u];
-    }
-    __syncwarp();
-    cluster_sync_all();                                // barrier 2: peers are done reading this CTA
-    // this owner's slice: [HA][dpo] f32 in sOwn, with (M, L) per head
-    const int64_t out_base = qi * HA * DV + static_cast<int64_t>(me) * dpo;
-    bool finish = p.ncl == 1;
-    if (p.ncl > 1) {
-      // publish the slice; the owner whose cluster arrives last merges them all
-      const int64_t slice = static_cast<int64_t>(dpo) * HA + 2 * HA;
-      float* g = p.part + ((qi * p.ncl + cl) * cs + me) * slice;
-      for (int i = et; i < dpo * HA / 4; i += 128)
-        reinterpret_cast<float4*>(g)[i] = reinterpret_cast<const float4*>(sOwn)[i];
-      if (et < HA) {
-        g[dpo * HA + et] = sMcl[et];
-        g[dpo * HA + HA + et] = sLcl[et];
-      }
-      __threadfence();
-      epi_bar();
-      if (et == 0) sh_ticket = atomicAdd(&p.ticket[qi * cs + me], 1u);
-      epi_bar();
-      finish = sh_ticket == static_cast<unsigned>(p.ncl - 1);
-      if (finish) {
+      tc_fence_before();
+      if (et == 0) {
+        bulk_wait_all();
+        fence_proxy_async_global();
         __threadfence();
-        const float* g0 = p.part + (qi * p.ncl * cs + me) * slice;   // cluster c2 at + c2*cs*slice
-        float* sWc = sML;                              // [ncl][HA] per-cluster weights ((m, l) exchange is over)
+      }
+      const int64_t base = buf + (blockIdx.x - tile);  // workspace slot of tile 0
+      const float* pb = p.part + base * kSlotFloats;   // slot j at pb + j * kSlotFloats
+      const int d0 = min(DV, tile * p.dpc), d1 = min(DV, d0 + p.dpc);
+      const uint32_t slice_bytes = static_cast<uint32_t>(d1 - d0) * HA * 4;
+      if (et == 0) {
+        // meet the query's other CTAs (all resident: the launch is cooperative)
+        unsigned long long* cnt = p.sync + slot;
+        const unsigned long long old = atomicAdd(cnt, 1ull);
+        const unsigned long long target = (old / p.T + 1) * p.T;
+        const uint64_t t0 = globaltimer_ns();
+        while (ld_acquire_u64(cnt) < target) {
+          if (globaltimer_ns() - t0 > 1000000000ull) {
+            raise_dev_error(p.err, DEVERR_TIMEOUT);
+            *abort_flag = 1;
+            break;
+          }
+        }
+        __threadfence();
+        fence_proxy_async_global();
+        if (p.bulk) {
+          // this CTA's dims of every partial into the KV region, every (m, l) into the P region
+          mbar_arrive_expect_tx(r_full, (slice_bytes + 2 * HA * 4) * p.T);
+          for (int j = 0; j < p.T; ++j) {
+            const float* sj = pb + static_cast<int64_t>(j) * kSlotFloats;
+            if (slice_bytes > 0) bulk_load(sKV + j * slice_bytes, sj + d0 * HA, slice_bytes, r_full);
+            bulk_load(sP + j * 2 * HA * 4, sj + kPartFloats, 2 * HA * 4, r_full);
+          }
+        }
+      }
+      epi_bar();
+      // weights of the T partials exp(m_j - M), the query's M and L
+      if (p.bulk) {
+        ok = mbar_wait(r_full, par, abort_flag, p.err) && ok;
+        if (et < HA) {
+          // T <= 32 here: all loads first, then the max, the weights and L in tile order
+          const uint32_t mlj = smem_u32(sP) + et * 4;  // m_j at + j*512, l_j at + j*512 + 256
+          float mj[32], lj[32];
+#pragma unroll
+          for (int j = 0; j < 32; ++j) {
+            mj[j] = j < p.T ? lds_f32(mlj + j * 2 * HA * 4) : -INFINITY;
+            lj[j] = j < p.T ? lds_f32(mlj + j * 2 * HA * 4 + HA * 4) : 0.0f;
+          }
+          float M = -INFINITY;
+#pragma unroll
+          for (int j = 0; j < 32; ++j) M = fmaxf(M, mj[j]);
+          float L = 0.0f;
+#pragma unroll
+          for (int j = 0; j < 32; ++j) {
+            const float wj = rescale(mj[j], M);
+            if (j < p.T) sW[j * HA + et] = wj;
+            L += lj[j] * wj;
+          }
+          sML2[et] = M;
+          sML2[HA + et] = L;
+        }
+      } else {
+        float* dstv = et < HA ? sW : sLv;                // m_j into sW, l_j into sLv
+#pragma unroll 8
+        for (int j = 0; j < p.T; ++j)
+          dstv[j * HA + (et & (HA - 1))] = __ldcg(pb + static_cast<int64_t>(j) * kSlotFloats + kPartFloats + et);
+        epi_bar();
         if (et < HA) {
           float M = -INFINITY;
-          for (int c2 = 0; c2 < p.ncl; ++c2) M = fmaxf(M, __ldcg(g0 + c2 * cs * slice + dpo * HA + et));
+          for (int j = 0; j < p.T; ++j) M = fmaxf(M, sW[j * HA + et]);
           float L = 0.0f;
-          for (int c2 = 0; c2 < p.ncl; ++c2) {
-            const float* gc = g0 + c2 * cs * slice;
-            const float wgt = rescale(__ldcg(gc + dpo * HA + et), M);
-            sWc[c2 * HA + et] = wgt;
-            L += __ldcg(gc + dpo * HA + HA + et) * wgt;
+          for (int j = 0; j < p.T; ++j) {
+            const float wj = rescale(sW[j * HA + et], M);
+            sW[j * HA + et] = wj;
+            L += sLv[j * HA + et] * wj;
           }
-          sMcl[et] = M;
-          sLcl[et] = L;
+          sML2[et] = M;
+          sML2[HA + et] = L;
+        }
+      }
+      epi_bar();
+      // this CTA's output dims: sum over the partials in tile order
+      const uint32_t w0 = smem_u32(sW);
+      for (int ds = d0; ds < d1; ds += kStageDims) {
+        const int nd = min(kStageDims, d1 - ds);
+        const int nch = nd * (HA / 4);                 // float4 chunks (dim, 4 heads)
+        for (int c0 = et; c0 < nch; c0 += 4 * 128) {
+          const int h4 = c0 & 15;                      // the same for every u below
+          uint32_t off[4];                             // byte offset of chunk u within a slice
+          bool in[4];
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const int c = c0 + u * 128;
+            const int dim = ds + (c >> 4);
+            in[u] = c < nch;
+            off[u] = static_cast<uint32_t>((dim - d0) * (HA * 4) + ((h4 ^ (dim & 7)) << 4));
+          }
+          float4 acc[4];
+#pragma unroll
+          for (int u = 0; u < 4; ++u) acc[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+          if (p.bulk) {
+#pragma unroll 4
+            for (int j = 0; j < p.T; ++j) {
+              float4 v[4];
+#pragma unroll
+              for (int u = 0; u < 4; ++u) v[u] = lds_v4f(kv0 + j * slice_bytes + (in[u] ? off[u] : 0));
+              const float4 wj = lds_v4f(w0 + (j * HA + 4 * h4) * 4);
+#pragma unroll
+              for (int u = 0; u < 4; ++u) {
+                acc[u].x += v[u].x * wj.x;
+                acc[u].y += v[u].y * wj.y;
+                acc[u].z += v[u].z * wj.z;
+                acc[u].w += v[u].w * wj.w;
+              }
+            }
+          } else {
+#pragma unroll 4
+            for (int j = 0; j < p.T; ++j) {
+              const uint8_t* sj = reinterpret_cast<const uint8_t*>(pb + static_cast<int64_t>(j) * kSlotFloats + d0 * HA);
+              float4 v[4];
+#pragma unroll
+              for (int u = 0; u < 4; ++u) v[u] = __ldcg(reinterpret_cast<const float4*>(sj + (in[u] ? off[u] : 0)));
+              const float4 wj = *reinterpret_cast<const float4*>(sW + j * HA + 4 * h4);
+#pragma unroll
+              for (int u = 0; u < 4; ++u) {
+                acc[u].x += v[u].x * wj.x;
+                acc[u].y += v[u].y * wj.y;
+                acc[u].z += v[u].z * wj.z;
+                acc[u].w += v[u].w * wj.w;
+              }
+            }
+          }
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            if (in[u]) {
+              const int dl = (c0 + u * 128) >> 4, h0 = 4 * h4;
+              sStage[(h0 + 0) * kStageStride + dl] = acc[u].x;
+              sStage[(h0 + 1) * kStageStride + dl] = acc[u].y;
+              sStage[(h0 + 2) * kStageStride + dl] = acc[u].z;
+              sStage[(h0 + 3) * kStageStride + dl] = acc[u].w;
+            }
+          }
         }
         epi_bar();
-        // 8 float4 chunks per thread and pass, two clusters per step: 16 loads in flight
-        const int nchunk = dpo * HA / 4;
-        for (int i0 = et; i0 < nchunk; i0 += 8 * 128) {
-          float4 acc[8];
-#pragma unroll
-          for (int u = 0; u < 8; ++u) acc[u] = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll 2
-          for (int c2 = 0; c2 < p.ncl; ++c2) {
-            const float4* gc = reinterpret_cast<const float4*>(g0 + c2 * cs * slice);
-            float4 v[8];
-#pragma unroll
-            for (int u = 0; u < 8; ++u) {
-              const int i = i0 + u * 128;
-              v[u] = i < nchunk ? __ldcg(gc + i) : make_float4(0.f, 0.f, 0.f, 0.f);
-            }
-#pragma unroll
-            for (int u = 0; u < 8; ++u) {
-              const int h = min((4 * (i0 + u * 128)) / dpo, HA - 1);
-              const float w = sWc[c2 * HA + h];
-              acc[u].x += v[u].x * w;
-              acc[u].y += v[u].y * w;
-              acc[u].z += v[u].z * w;
-              acc[u].w += v[u].w * w;
-            }
-          }
-#pragma unroll
-          for (int u = 0; u < 8; ++u) {
-            const int i = i0 + u * 128;
-            if (i < nchunk) reinterpret_cast<float4*>(sOwn)[i] = acc[u];
-          }
+        if (more && ds + kStageDims >= d1) issue_gather(qi + p.G);   // the KV region is free again
+        // normalise, bf16, 8-byte stores of 4 dims
+        const int pieces = nd / 4;
+        for (int i = et; i < HA * pieces; i += 128) {
+          const int h = i / pieces, pc = i % pieces;
+          const float L = sML2[HA + h];
+          const float inv = L > 0.0f ? 1.0f / L : 0.0f;
+          const float* a = sStage + h * kStageStride + 4 * pc;
+          uint2 o;
+          o.x = pack_bf16x2(a[0] * inv, a[1] * inv);
+          o.y = pack_bf16x2(a[2] * inv, a[3] * inv);
+          *reinterpret_cast<uint2*>(p.out + (qi * HA + h) * DV + ds + 4 * pc) = o;
         }
-        if (et == 0) p.ticket[qi * cs + me] = 0u;     // ready for the next call
         epi_bar();
       }
-    }
-    if (finish) {
-      // normalise, bf16, coalesced 16-byte stores of the owned [64 heads x dpo dims] block
-      const int pieces = dpo / 8;
-      for (int i = et; i < HA * pieces; i += 128) {
-        const int h = i / pieces, pc = i % pieces;
-        const float L = sLcl[h];
-        const float inv = L > 0.0f ? 1.0f / L : 0.0f;
-        const float* a = sOwn + h * dpo + pc * 8;
-        uint4 o;
-        o.x = pack_bf16x2(a[0] * inv, a[1] * inv);
-        o.y = pack_bf16x2(a[2] * inv, a[3] * inv);
-        o.z = pack_bf16x2(a[4] * inv, a[5] * inv);
-        o.w = pack_bf16x2(a[6] * inv, a[7] * inv);
-        *reinterpret_cast<uint4*>(p.out + out_base + static_cast<int64_t>(h) * DV + pc * 8) = o;
+      if (more && d1 <= d0) issue_gather(qi + p.G);
+      if (tile == 0 && p.lse && et < HA)
+        p.lse[qi * HA + et] = sML2[HA + et] > 0.0f ? sML2[et] + logf(sML2[HA + et]) : -INFINITY;
+      // this CTA alone reads its dims of every partial: drop those lines from L2
+      if (d1 > d0) {
+        const int lines = static_cast<int>(slice_bytes / 128);
+        for (int i = et; i < p.T * lines; i += 128) {
+          const int j = i / lines, ln = i % lines;
+          discard_l2_line(pb + static_cast<int64_t>(j) * kSlotFloats + d0 * HA + ln * 32);
+        }
       }
-      if (me == 0 && p.lse && et < HA)
-        p.lse[qi * HA + et] = sLcl[et] > 0.0f ? sMcl[et] + logf(sLcl[et]) : -INFINITY;
+      epi_bar();
+      if (et == 0) mbar_arrive(m_done);
+      if (more) publish_gather();
     }
+    cp_async_wait<0>();
   }
 
   // ---------------------------------------------------------------- teardown
-  if (threadIdx.x == 32) {
-    // loads may still be landing if a wait gave up early (bounded: 0.1 s)
-    const uint64_t t0 = globaltimer_ns();
-    while (!mbar_try_wait(q_full, 0) && globaltimer_ns() - t0 < 100000000ull) {
-    }
-    for (int kb = 0; kb < kKB; ++kb)
-      while (!mbar_try_wait(&kv_full[kb], 0) && globaltimer_ns() - t0 < 100000000ull) {
-      }
-  }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -483,105 +574,122 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 struct Shape {
-  int cs, ncl;
+  int T, dpc;
 };
 
-// Cluster size and clusters per query for k selected rows (depends on k only).
 Shape shape_for(int k) {
-  const int tiles = (k + kRows - 1) / kRows;
-  // Clusters of 4 leave every cluster of a batch-8 decode co-resident; of 8,
-  // fewer fit at once than 148 SMs would suggest (whole GPCs are needed).
-  int max_cs = kDefaultCS;
-  if (const char* e = getenv("CSA2_ATTN_MAX_CLUSTER")) {   // tests: other cluster sizes
+  const int T = (k + kRows - 1) / kRows;
+  const int per = (DV + T - 1) / T;
+  return {T, (per + 3) / 4 * 4};
+}
+
+// CTAs of this kernel that fit on the device at once (cached), capped by the
+// environment variable CSA2_ATTN_MAX_CTAS (tests: several waves per launch).
+int resident_ctas() {
+  static std::once_flag once;
+  static int cap = 0;
+  std::call_once(once, [] {
+    int per_sm = 0;
+    if (cudaFuncSetAttribute(attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES) !=
+            cudaSuccess ||
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, attn_tc_kernel, kThreads, SMEM_BYTES) !=
+            cudaSuccess) {
+      cudaGetLastError();
+      per_sm = 0;
+    }
+    cap = std::min(per_sm * sm_count(), kAttnMaxGrid);
+  });
+  int c = cap;
+  if (const char* e = getenv("CSA2_ATTN_MAX_CTAS")) {
     const int v = atoi(e);
-    if (v == 2 || v == 4 || v == 8) max_cs = v;
-    if (v == 1) max_cs = kMinCS;
+    if (v > 0) c = std::min(c, v);
   }
-  int cs = kMinCS;
-  while (cs < tiles && cs < max_cs) cs *= 2;
-  return {cs, (tiles + cs - 1) / cs};
-}
-
-size_t part_bytes(int64_t n_queries, Shape s) {
-  if (s.ncl <= 1) return 0;
-  const int64_t slice = static_cast<int64_t>(DV / s.cs) * HA + 2 * HA;
-  return static_cast<size_t>(n_queries * s.ncl * s.cs * slice * 4);
-}
-
-size_t ticket_bytes(int64_t n_queries, Shape s) {
-  return s.ncl <= 1 ? 0 : static_cast<size_t>(n_queries * s.cs * 4);
+  return c;
 }
 
 size_t a256(size_t x) { return (x + 255) & ~size_t(255); }
 
+// Workspace sized for the largest grid the kernel can get on any device
+// (kAttnMaxGrid CTAs), so that its size does not depend on the device.
+struct WsLayout {
+  size_t part, sync, total;
+};
+WsLayout ws_layout(int64_t n_queries, Shape s) {
+  const int64_t g = std::min<int64_t>(n_queries, kAttnMaxGrid / s.T);
+  const int64_t ctas = g * s.T;
+  WsLayout l;
+  l.part = a256(static_cast<size_t>(2 * ctas) * kSlotFloats * 4);
+  l.sync = a256(static_cast<size_t>(g) * 8);
+  l.total = l.part + l.sync;
+  return l;
+}
+
+bool applies(int Ha, int D, int k, csa2_kv_fmt fmt) {
+  if (fmt != CSA2_KV_BF16 || Ha != HA || D != DV || k <= 0) return false;
+  const Shape s = shape_for(k);
+  return s.T <= kMaxTiles && s.T <= kAttnMaxGrid;
+}
+
 }  // namespace
 
 size_t sparse_attn_tc_workspace(int B, int Q, int Ha, int D, int k, csa2_kv_fmt fmt) {
-  if (fmt != CSA2_KV_BF16 || Ha != HA || D != DV || k <= 0) return 0;
-  const Shape s = shape_for(k);
-  const int64_t nq = static_cast<int64_t>(B) * Q;
-  if (s.ncl <= 1 || s.ncl > kMaxNCL) return 0;
-  return a256(part_bytes(nq, s)) + a256(ticket_bytes(nq, s));
+  if (!applies(Ha, D, k, fmt)) return 0;
+  return ws_layout(static_cast<int64_t>(B) * Q, shape_for(k)).total;
 }
 
 csa2_status launch_sparse_attn_tc(const void* q, const csa2_kv& kv, const int32_t* topk, int B,
                                   int Q, int Ha, int k, float scale, void* out, float* lse,
-                                  void* ws, size_t ws_bytes, cudaStream_t stream) {
+                                  void* ws, size_t ws_bytes, unsigned long long* sync_zeroed,
+                                  cudaStream_t stream) {
   if (getenv("CSA2_ATTN_SIMT")) return CSA2_ERR_UNSUPPORTED;      // force the CUDA-core kernel
-  if (kv.fmt != CSA2_KV_BF16 || kv.dim != DV || Ha != HA || k <= 0) return CSA2_ERR_UNSUPPORTED;
+  if (!applies(Ha, kv.dim, k, kv.fmt)) return CSA2_ERR_UNSUPPORTED;
   const int64_t n_queries = static_cast<int64_t>(B) * Q;
-  if (n_queries * HA > 0x7fffffffLL || static_cast<int64_t>(B) * kv.n > 0x7fffffffLL)
-    return CSA2_ERR_UNSUPPORTED;
+  if (n_queries * HA > 0x7fffffffLL) return CSA2_ERR_UNSUPPORTED;
   const Shape s = shape_for(k);
-  if (s.ncl > kMaxNCL || n_queries * s.cs * s.ncl > 0x7fffffffLL) return CSA2_ERR_UNSUPPORTED;
-  const size_t need = sparse_attn_tc_workspace(B, Q, Ha, kv.dim, k, kv.fmt);
-  if (need > 0 && (!ws || ws_bytes < need)) return CSA2_ERR_UNSUPPORTED;
-  CUtensorMap qmap, kvmap;
+  const int cap = resident_ctas();
+  if (cap < s.T) return CSA2_ERR_UNSUPPORTED;
+  const WsLayout lay = ws_layout(n_queries, s);
+  if (!ws || ws_bytes < lay.total) return CSA2_ERR_UNSUPPORTED;
+  const int64_t G = std::min<int64_t>(n_queries, cap / s.T);
+  CUtensorMap qmap;
   memset(&qmap, 0, sizeof(qmap));
-  memset(&kvmap, 0, sizeof(kvmap));
   CSA2_TRY(make_tensor_map_bf16_2d(&qmap, q, static_cast<uint64_t>(n_queries) * HA, DV, DV * 2, 64, HA));
-  CSA2_TRY(make_tensor_map_bf16_2d(&kvmap, kv.data, static_cast<uint64_t>(B) * kv.n, DV, DV * 2, 64, 1));
   Params p;
   p.topk = topk;
+  p.kv = static_cast<const uint16_t*>(kv.data);
   p.out = static_cast<uint16_t*>(out);
   p.lse = lse;
-  p.part = nullptr;
-  p.ticket = nullptr;
-  if (s.ncl > 1) {
-    p.part = static_cast<float*>(ws);
-    p.ticket = reinterpret_cast<unsigned*>(static_cast<char*>(ws) + a256(part_bytes(n_queries, s)));
-    begin_launch(stream);
-    if (cudaMemsetAsync(p.ticket, 0, ticket_bytes(n_queries, s), stream) != cudaSuccess)
-      return check_launch("sparse_attn_tc: clear tickets");
-    note_launch(LK_OTHER, 1, stream);
-  }
+  p.part = static_cast<float*>(ws);
+  p.sync = sync_zeroed ? sync_zeroed
+                       : reinterpret_cast<unsigned long long*>(static_cast<char*>(ws) + lay.part);
   p.err = device_error_word();
   p.n = kv.n;
+  p.n_queries = n_queries;
   p.Q = Q;
   p.k = k;
-  p.cs = s.cs;
-  p.ncl = s.ncl;
+  p.T = s.T;
+  p.G = static_cast<int>(G);
+  p.dpc = s.dpc;
+  p.bulk = static_cast<int64_t>(s.T) * s.dpc * HA * 4 <= kKB * kKBBytes && s.T * 2 * HA * 4 <= kRows * 128;
   p.scale = scale;
-  static std::once_flag once;
-  static cudaError_t attr = cudaSuccess;
-  std::call_once(once, [] {
-    attr = cudaFuncSetAttribute(attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
-  });
-  if (attr != cudaSuccess) return fail(CSA2_ERR_CUDA, "sparse_attn_tc: function attributes");
+  if (!sync_zeroed) {          // a caller workspace: counters start at zero
+    begin_launch(stream);
+    if (cudaMemsetAsync(p.sync, 0, static_cast<size_t>(G) * 8, stream) != cudaSuccess)
+      return check_launch("sparse_attn_tc: clear counters");
+    note_launch(LK_OTHER, 1, stream);
+  }
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(static_cast<unsigned>(n_queries * s.cs * s.ncl));
+  cfg.gridDim = dim3(static_cast<unsigned>(G * s.T));
   cfg.blockDim = dim3(kThreads);
   cfg.dynamicSmemBytes = SMEM_BYTES;
   cfg.stream = stream;
   cudaLaunchAttribute at[1];
-  at[0].id = cudaLaunchAttributeClusterDimension;
-  at[0].val.clusterDim.x = s.cs;
-  at[0].val.clusterDim.y = 1;
-  at[0].val.clusterDim.z = 1;
+  at[0].id = cudaLaunchAttributeCooperative;
+  at[0].val.cooperative = 1;
   cfg.attrs = at;
   cfg.numAttrs = 1;
   begin_launch(stream);
-  const cudaError_t e = cudaLaunchKernelEx(&cfg, attn_tc_kernel, qmap, kvmap, p);
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, attn_tc_kernel, qmap, p);
   note_launch(LK_ATTN, 1, stream);
   if (e != cudaSuccess) {
     cudaGetLastError();

@@ -29,6 +29,7 @@ struct csa2_group {
   int32_t* pool = nullptr;   // [B, Q, P]   pool of the last Full layer (P > 0)
   void* ws = nullptr;        // scores + selection state, then attention workspace
   size_t ws_bytes = 0;
+  unsigned long long* attn_sync = nullptr;  // attention arrival counters, zeroed once
   bool have_full = false;
   csa2_kv kv{};              // registered by the last Full layer (not owned)
   const void* index_k = nullptr;
@@ -70,6 +71,8 @@ csa2_status csa2_group_create(csa2_group** group, const csa2_group_desc* d) {
   cudaError_t e = cudaMalloc(&g->topk, a256(rows * d->k * sizeof(int32_t)));
   if (e == cudaSuccess && d->P > 0) e = cudaMalloc(&g->pool, a256(rows * d->P * sizeof(int32_t)));
   if (e == cudaSuccess) e = cudaMalloc(&g->ws, g->ws_bytes);
+  if (e == cudaSuccess) e = cudaMalloc(&g->attn_sync, kAttnMaxGrid * sizeof(unsigned long long));
+  if (e == cudaSuccess) e = cudaMemset(g->attn_sync, 0, kAttnMaxGrid * sizeof(unsigned long long));
   if (e != cudaSuccess) {
     cudaGetLastError();
     csa2_group_destroy(g);
@@ -87,6 +90,7 @@ void csa2_group_destroy(csa2_group* g) {
   if (g->topk) cudaFree(g->topk);
   if (g->pool) cudaFree(g->pool);
   if (g->ws) cudaFree(g->ws);
+  if (g->attn_sync) cudaFree(g->attn_sync);
   cudaSetDevice(prev);
   delete g;
 }
@@ -149,8 +153,9 @@ csa2_status csa2_group_layer(csa2_group* g, int layer, const csa2_layer_io* io,
                         d.P, d.k, g->topk, nullptr, 0, d.act, g->ws, g->ws_bytes, stream);
     if (s != CSA2_OK) return s;
   }
-  return csa2_sparse_attn(mode, io->q_attn, &g->kv, g->topk, d.B, d.Q, d.Ha, d.k, d.scale, io->out,
-                          io->lse, g->ws, g->ws_bytes, stream);
+  return sparse_attn_checked(mode, io->q_attn, &g->kv, g->topk, d.B, d.Q, d.Ha, d.k, d.scale,
+                             io->out, io->lse, g->ws, g->ws_bytes, g->attn_sync,
+                             reinterpret_cast<cudaStream_t>(stream));
 }
 
 }  // extern "C"

@@ -21,14 +21,33 @@ size_t select_topk_workspace(int64_t rows, int64_t L, int count);
 csa2_status launch_select_topk2(const float* scores, int64_t rows, int64_t L, int count0,
                                 const int32_t* ids, int32_t* out0, int count1, int32_t* out1,
                                 void* ws, size_t ws_bytes, cudaStream_t stream);
+// One CTA per row, no workspace: rows of up to kSelectCtaMaxL scores.
+constexpr int64_t kSelectCtaMaxL = 32768;
+bool select_topk_cta_applies(int64_t rows, int64_t L);
+csa2_status launch_select_topk_cta(const float* scores, int64_t rows, int64_t L, int count0,
+                                   const int32_t* ids, int32_t* out0, int count1, int32_t* out1,
+                                   cudaStream_t stream);
 csa2_status launch_select_topk(const float* scores, int64_t rows, int64_t L, int count,
                                const int32_t* ids, int32_t* out, void* ws, size_t ws_bytes,
                                cudaStream_t stream);
 
+// Largest grid of the tensor-core attention kernel on any device (>= the
+// CTAs that fit at once); sizes its workspace and its arrival counters.
+constexpr int kAttnMaxGrid = 160;
+
 size_t sparse_attn_workspace(int B, int Q, int Ha, int D, int k, csa2_kv_fmt fmt);
+// sync_zeroed: kAttnMaxGrid arrival counters that were zero before their
+// first use and are left consistent by every launch (a layer group's), or
+// NULL to take them from the workspace and clear them on the stream.
 csa2_status launch_sparse_attn(const void* q, const csa2_kv& kv, const int32_t* topk, int B,
                                int Q, int Ha, int k, float scale, void* out, float* lse, void* ws,
-                               size_t ws_bytes, cudaStream_t stream);
+                               size_t ws_bytes, unsigned long long* sync_zeroed,
+                               cudaStream_t stream);
+// csa2_sparse_attn's argument checks, then launch_sparse_attn.
+csa2_status sparse_attn_checked(csa2_mode mode, const void* q, const csa2_kv* kv,
+                                const int32_t* topk, int B, int Q, int Ha, int k, float scale,
+                                void* out, float* lse, void* workspace, size_t workspace_bytes,
+                                unsigned long long* sync_zeroed, cudaStream_t stream);
 
 csa2_status launch_fp4_pack(const void* x, int64_t rows, int D, uint8_t* codes, uint8_t* scales,
                             cudaStream_t stream);

@@ -33,8 +33,9 @@ constexpr int kT = 1024;
 // Order-preserving key: larger score -> larger key.  -inf and NaN map to 0,
 // which no selectable score has (the smallest valid key is 0x00800000).
 __device__ __forceinline__ uint32_t score_key(float f) {
-  const uint32_t u = __float_as_uint(f);
+  uint32_t u = __float_as_uint(f);
   if (f != f || u == 0xff800000u) return 0u;
+  if (u == 0x80000000u) u = 0u;                    // -0 ranks as +0
   return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 

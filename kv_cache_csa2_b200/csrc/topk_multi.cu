@@ -58,8 +58,9 @@ struct SelParams {
 };
 
 __device__ __forceinline__ uint32_t score_key(float f) {
-  const uint32_t u = __float_as_uint(f);
+  uint32_t u = __float_as_uint(f);
   if (f != f || u == 0xff800000u) return 0u;
+  if (u == 0x80000000u) u = 0u;                    // -0 ranks as +0
   return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
@@ -415,8 +416,14 @@ int max_resident_ctas(size_t smem) {
   return per_sm_cache[slot] * sm_count();
 }
 
+// The one-CTA kernel of topk_cta.cu takes rows of up to kSelectCtaMaxL keys
+// unless CSA2_TOPK_NO_CTA is set (tests: this kernel's one-chunk path).
+bool cta_kernel_takes(int64_t rows, int64_t L) {
+  return select_topk_cta_applies(rows, L) && !getenv("CSA2_TOPK_NO_CTA");
+}
+
 bool multi_applies(int64_t rows, int64_t L) {
-  if (getenv("CSA2_TOPK_ONE_CTA")) return false;
+  if (getenv("CSA2_TOPK_ONE_CTA") || cta_kernel_takes(rows, L)) return false;
   if (rows <= 0 || rows > kMaxRowsMulti || L < 2048) return false;
   const int64_t C = (L + chunk_for(L) - 1) / chunk_for(L);
   return C <= kMaxC;
@@ -437,6 +444,8 @@ size_t select_topk_multi_workspace(int64_t rows, int64_t L, int) {
 csa2_status launch_select_topk2(const float* scores, int64_t rows, int64_t L, int count0,
                                 const int32_t* ids, int32_t* out0, int count1, int32_t* out1,
                                 void* ws, size_t ws_bytes, cudaStream_t stream) {
+  if (cta_kernel_takes(rows, L))
+    return launch_select_topk_cta(scores, rows, L, count0, ids, out0, count1, out1, stream);
   if (!multi_applies(rows, L)) return CSA2_ERR_UNSUPPORTED;
   const int chunk = chunk_for(L);
   const int C = static_cast<int>((L + chunk - 1) / chunk);

@@ -181,6 +181,7 @@ def _score_rows(r, rows, L, kind):
 
 
 @pytest.mark.parametrize("rows,L,count", [(5, 1000, 37), (3, 4096, 2048), (2, 300, 1000), (1, 1, 1),
+                                          (8, 16384, 2048), (2, 32768, 16384), (3, 20001, 5000),
                                           (4, 70000, 2048), (2, 262144, 16384), (64, 2000, 256)])
 @pytest.mark.parametrize("kind", ["normal", "ties"])
 def test_select_topk_exact(rows, L, count, kind):
@@ -190,6 +191,28 @@ def test_select_topk_exact(rows, L, count, kind):
     s64 = np.where(np.isnan(s), -np.inf, s).astype(np.float64)
     want = O.select_top(s64, count)
     assert np.array_equal(got, want)
+
+
+@pytest.mark.parametrize("rows,L,count", [(3, 4096, 2048), (8, 16384, 2048), (2, 32768, 16384)])
+def test_select_topk_chunked_path(rows, L, count, monkeypatch):
+    """Rows up to 32768 scores normally take the one-CTA kernel; the
+    cooperative kernel's one-chunk path gives the same result."""
+    monkeypatch.setenv("CSA2_TOPK_NO_CTA", "1")
+    r = _rng(17)
+    s = _score_rows(r, rows, L, "ties")
+    got = K.csa2_select_topk(U.dev(s), count).cpu().numpy()
+    want = O.select_top(np.where(np.isnan(s), -np.inf, s).astype(np.float64), count)
+    assert np.array_equal(got, want)
+
+
+@pytest.mark.parametrize("L", [3000, 100000])
+def test_select_topk_signed_zero_ties(L):
+    """-0 and +0 are the same score: ties between them go to the lower position."""
+    r = _rng(18)
+    s = np.where(r.random((2, L)) < 0.5, np.float32(0.0), np.float32(-0.0)).astype(np.float32)
+    s[:, ::7] = 1.0
+    got = K.csa2_select_topk(U.dev(s), L // 2).cpu().numpy()
+    assert np.array_equal(got, O.select_top(s.astype(np.float64), L // 2))
 
 
 def test_select_topk_maps_ids():
@@ -237,17 +260,22 @@ def test_sparse_attn_parity(Ha, D, N, k, fp4):
     U.check_attn(U.host_bf16(out), lse.cpu().numpy().astype(np.float64), o, l, f"Ha{Ha} D{D} k{k}")
 
 
-@pytest.mark.parametrize("max_cluster", ["1", "2", "4", "8"])
-def test_sparse_attn_smaller_clusters(max_cluster, monkeypatch):
-    """The tensor-core kernel splits a query over a cluster of CTAs; smaller
-    clusters give each CTA more tiles (re-gathered for the PV product)."""
-    monkeypatch.setenv("CSA2_ATTN_MAX_CLUSTER", max_cluster)
+@pytest.mark.parametrize("max_ctas,k", [("8", 384), ("8", 1000), ("16", 1000), ("40", 1000)])
+def test_sparse_attn_grid_waves(max_ctas, k, monkeypatch):
+    """The tensor-core kernel runs a grid of whole queries (one CTA per
+    128-row tile) and loops over the batch in waves; a smaller grid means more
+    waves, with the same reduction order and so the same bits."""
     r = _rng(19)
-    B, Q, Ha, D, N, k = 2, 2, 64, 512, 4000, 384 if max_cluster == "1" else 1000
+    B, Q, Ha, D, N = 2, 3, 64, 512, 4000
     q, kv, topk = _attn_case(r, B, Q, Ha, D, N, k, False)
-    out, lse = K.csa2_sparse_attn(U.dev_bf16(q), U.dev_bf16(kv), U.dev(topk), D ** -0.5)
+    args = (U.dev_bf16(q), U.dev_bf16(kv), U.dev(topk), D ** -0.5)
+    full_out, full_lse = K.csa2_sparse_attn(*args)
+    monkeypatch.setenv("CSA2_ATTN_MAX_CTAS", max_ctas)
+    for _ in range(2):                       # twice in a row
+        out, lse = K.csa2_sparse_attn(*args)
+        assert torch.equal(out, full_out) and torch.equal(lse, full_lse)
     o, _, l = O.sparse_attn(O.bf16_bits_to_float(q), O.bf16_bits_to_float(kv), topk, D ** -0.5)
-    U.check_attn(U.host_bf16(out), lse.cpu().numpy().astype(np.float64), o, l, f"cluster<={max_cluster}")
+    U.check_attn(U.host_bf16(out), lse.cpu().numpy().astype(np.float64), o, l, f"ctas<={max_ctas}")
 
 
 def test_sparse_attn_bounds_recorded_not_faulting():
