@@ -156,7 +156,8 @@ def source_digest(*names) -> str:
 PROFILED_SOURCES = {
     "index_scores": (("index_scores.cu", "index_scores_tc.cu"), "profiles/index_scores_c4.md"),
     "attn": (("attn.cu", "attn_tc.cu"), "profiles/attn_c4.md"),
-    "topk": (("topk.cu", "topk_multi.cu"), "profiles/topk_c4.md"),
+    "topk": (("topk.cu", "topk_multi.cu", "topk_cta.cu"), "profiles/topk_c4.md"),
+    "index_pool": (("index_scores.cu", "index_scores_tc.cu"), "profiles/index_pool_c4.md"),
 }
 
 
@@ -475,11 +476,22 @@ def oracle_queries(wl, inp, queries):
     from kv_cache_csa2_b200 import inputs as I
 
     t0 = time.perf_counter()
+    n_cached = inp["kv"].shape[1]
     for b, t in queries:
         kb = inp["kv"][b:b + 1]
+        new = None
+        if wl.compress_new_tokens:         # the newest entries come from raw tokens: compress them
+            _, new = O.compress(O.bf16_bits_to_float(inp["c"][b:b + 1]),
+                                inp["z"][b:b + 1].astype(np.float64),
+                                inp["bias"].astype(np.float64), wl.m, wl.halo)
 
-        def rows(_, ids, kb=kb):
-            r = O.bf16_bits_to_float(kb[0, ids])
+        def rows(_, ids, kb=kb, new=new):
+            ids = np.asarray(ids)
+            r = np.empty((len(ids), wl.D))
+            old = ids < n_cached
+            r[old] = O.bf16_bits_to_float(kb[0, ids[old]])
+            if (~old).any():
+                r[~old] = new[0, ids[~old] - n_cached]
             return O.fp4_unpack(*O.fp4_pack(r)) if wl.kv_fp4 else r
 
         layers = []
@@ -542,6 +554,45 @@ def run_reference(args, wl, world, rank):
                     "d2h_bytes_per_step": 0}}
 
 
+# ---------------------------------------------------------------------------- kernel cases
+
+def run_kernel_case(name, reps=4):
+    """One library call of the c4 group on seeded synthetic inputs, `reps` times
+    (a short program for ncu captures of one kernel; prints one JSON line).
+      attn     csa2_sparse_attn, 8 queries x 64 heads x 512, k = 2048, 32768
+               entries per sequence (the kernel gathers 2048 rows either way)
+      full     csa2_index_topk(FULL) over 8 x 262144 entries, pool 16384 + top 2048
+      reindex  csa2_index_topk(REINDEX) inside a 16384-slot pool, top 2048"""
+    import torch
+    import kv_cache_csa2_b200 as K
+    g = torch.Generator(device="cuda").manual_seed(0)
+    B = 8
+    if name == "attn":
+        N, D, Ha, k = 32768, 512, 64, 2048
+        kv = torch.randn(B, N, D, device="cuda", generator=g).to(torch.bfloat16)
+        q = torch.randn(B, 1, Ha, D, device="cuda", generator=g).to(torch.bfloat16)
+        ids = torch.stack([torch.sort(torch.randperm(N, device="cuda", generator=g)[:k])[0] for _ in range(B)])
+        topk = ids.view(B, 1, k).to(torch.int32)
+        for _ in range(reps):
+            K.csa2_sparse_attn(q, kv, topk, D ** -0.5)
+    else:
+        N = 262144
+        q = (torch.randn(B, 1, 64, 128, device="cuda", generator=g) / 11.3).to(torch.bfloat16)
+        w = torch.rand(B, 1, 64, device="cuda", generator=g)
+        k = (torch.randn(B, N, 128, device="cuda", generator=g) / 11.3).to(torch.bfloat16)
+        if name == "full":
+            for _ in range(reps):
+                K.csa2_index_topk(K.FULL, q, w, k, 2048, pool_size=16384)
+        else:
+            ids = torch.stack([torch.sort(torch.randperm(N, device="cuda", generator=g)[:16384])[0] for _ in range(B)])
+            pool = ids.view(B, 1, 16384).to(torch.int32)
+            for _ in range(reps):
+                K.csa2_index_topk(K.REINDEX, q, w, k, 2048, pool_in=pool)
+    torch.cuda.synchronize()
+    K.csa2_device_error()
+    return {"kernel_case": name, "reps": reps, "ok": True}
+
+
 # ---------------------------------------------------------------------------- main
 
 def main(argv=None):
@@ -555,7 +606,12 @@ def main(argv=None):
     ap.add_argument("--cpu-budget", type=float, default=20.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--eager", action="store_true", help="launch layers eagerly instead of CUDA graphs")
+    ap.add_argument("--kernel-case", choices=["attn", "full", "reindex"],
+                    help="run one library call of the group 4 times and exit (for ncu captures)")
     args = ap.parse_args(argv)
+    if args.kernel_case:
+        print(json.dumps(run_kernel_case(args.kernel_case)), flush=True)
+        return
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     from kv_cache_csa2_b200.configs import CONFIGS

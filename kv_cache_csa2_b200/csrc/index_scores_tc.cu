@@ -7,10 +7,11 @@
 // padded heads are zero) by d (MMA K, 16 per instruction).  Per CTA
 // (persistent, one per SM):
 //   warp 0     producer: per tile, the 128 key rows into a shared-memory ring
-//              (dense: two TMA tiled loads per 128-column K-block; pool: a
-//              cp.async gather of the rows the pool names, zero-filled for
-//              empty slots); per query group, the queries (swizzled) and head
-//              weights into one of two slots;
+//              (dense: one TMA tiled load per 64-column K-block; pool: a
+//              cp.async gather of the rows the pool names by warps 0, 6, 7, 8,
+//              zero-filled for empty slots); per query group, the queries
+//              (TMA when a group is one query of unpadded heads, else swizzled
+//              by the lanes) and head weights into one of two slots;
 //   warp 1     allocates TMEM; one lane issues the MMAs of a tile into one of
 //              two accumulators and commits them to the ring slot and the
 //              accumulator barriers;
@@ -38,7 +39,7 @@ constexpr int kThreads = kWarps * 32;
 constexpr int kPoolThreads = 9 * 32;
 constexpr int kTileRows = 128;
 constexpr int kKBlockBytes = kTileRows * 128;  // 128 rows x 64 bf16
-constexpr int kLag = 2;                        // pool gathers: stages of copies kept in flight
+constexpr int kLag = 3;                        // pool gathers: stages of copies kept in flight
 
 struct Params {
   const uint16_t* q;
@@ -51,6 +52,7 @@ struct Params {
   int Q, H, P;
   int64_t N;
   int relu;
+  int q_tma;          // queries by TMA (one query per group, no padded heads)
   int n_qgroups, n_tiles;
   int64_t n_units;
 };
@@ -80,7 +82,8 @@ struct Cfg {
 
 template <int DK, int NQ, int HP, bool POOL>
 __global__ void __launch_bounds__(POOL ? kPoolThreads : kThreads, 1)
-    index_tc_kernel(const __grid_constant__ CUtensorMap kmap, const Params p) {
+    index_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap qmap,
+                    const Params p) {
   using C = Cfg<DK, NQ, HP, POOL>;
   constexpr int S = C::STAGES;
   extern __shared__ uint8_t smem_raw[];
@@ -119,6 +122,7 @@ __global__ void __launch_bounds__(POOL ? kPoolThreads : kThreads, 1)
     *abort_flag = 0;
     fence_mbar_init();
     if (!POOL) prefetch_tensor_map(&kmap);
+    if (p.q_tma) prefetch_tensor_map(&qmap);
   }
   if (warp == 1) {
     tmem_alloc(tmem_slot, C::TMEM_COLS);
@@ -136,6 +140,21 @@ __global__ void __launch_bounds__(POOL ? kPoolThreads : kThreads, 1)
     int qi = -1;
     int64_t it = 0;
     bool ok = true;
+    // pool gather: thread ptid copies 16-byte chunk c16 of rows rg + 16 i
+    // (i < 8) in every K-block, so eight consecutive lanes read one 128-byte
+    // segment; the ids of the next unit are loaded during the current one
+    const int c16 = ptid & 7, rg = ptid >> 3;
+    auto pool_ids = [&](int64_t v, int32_t (&ids)[8]) {
+      const int64_t bgv = v / p.n_tiles;
+      const int64_t qrow = (bgv / p.n_qgroups) * p.Q + bgv % p.n_qgroups;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const int64_t slot_i = (v % p.n_tiles) * kTileRows + rg + 16 * i;
+        ids[i] = slot_i < L ? p.pool[qrow * p.P + slot_i] : -1;
+      }
+    };
+    int32_t next_ids[8];
+    if (POOL && u0 < u1) pool_ids(u0, next_ids);
     for (int64_t u = u0; u < u1 && ok; ++u, ++it) {
       const int64_t bg = u / p.n_tiles;
       const int t = static_cast<int>(u % p.n_tiles);
@@ -149,15 +168,41 @@ __global__ void __launch_bounds__(POOL ? kPoolThreads : kThreads, 1)
         const int slot = qi & 1;
         if (qi >= 2 && !mbar_wait(&qempty[slot], ((qi >> 1) - 1) & 1, abort_flag, p.err)) { ok = false; break; }
         uint8_t* qs = sQ + slot * C::QBYTES;
-        // rows r = qq * HP + h; 16-byte chunks c = kb * 8 + cc
-        for (int i = lane; i < C::QROWS * (DK / 8); i += 32) {
-          const int r = i / (DK / 8), c = i % (DK / 8);
-          const int qq = r / HP, h = r % HP;
-          const int query = g * NQ + qq;
-          uint4 v = make_uint4(0, 0, 0, 0);
-          if (h < p.H && query < p.Q)
-            v = *reinterpret_cast<const uint4*>(p.q + ((static_cast<int64_t>(b) * p.Q + query) * p.H + h) * DK + c * 8);
-          *reinterpret_cast<uint4*>(qs + (c / 8) * C::QKB + sw128_offset(r, c % 8)) = v;
+        if (p.q_tma) {
+          // head weights by the lanes, then the query's HP x DK heads by TMA
+          for (int r = lane; r < C::QROWS; r += 32)
+            sW[slot * C::QROWS + r] = p.w[(static_cast<int64_t>(b) * p.Q + g) * p.H + r];
+          __syncwarp();
+          if (lane == 0) {
+            mbar_arrive_expect_tx(&qfull[slot], C::QBYTES);
+#pragma unroll
+            for (int kb = 0; kb < C::KB; ++kb)
+              tma_load_2d(qs + kb * C::QKB, &qmap, &qfull[slot], kb * 64,
+                          static_cast<int32_t>((static_cast<int64_t>(b) * p.Q + g) * p.H));
+          }
+          prev_bg = bg;
+        } else {
+        // rows r = qq * HP + h; 16-byte chunks c = kb * 8 + cc; 8 loads per
+        // lane in flight before any is stored
+        constexpr int NCH = C::QROWS * (DK / 8);
+        for (int i0 = lane; i0 < NCH; i0 += 32 * 8) {
+          uint4 v[8];
+#pragma unroll
+          for (int u = 0; u < 8; ++u) {
+            const int i = i0 + 32 * u;
+            const int r = i / (DK / 8), c = i % (DK / 8);
+            const int qq = r / HP, h = r % HP;
+            const int query = g * NQ + qq;
+            v[u] = make_uint4(0, 0, 0, 0);
+            if (i < NCH && h < p.H && query < p.Q)
+              v[u] = __ldg(reinterpret_cast<const uint4*>(p.q + ((static_cast<int64_t>(b) * p.Q + query) * p.H + h) * DK + c * 8));
+          }
+#pragma unroll
+          for (int u = 0; u < 8; ++u) {
+            const int i = i0 + 32 * u;
+            const int r = i / (DK / 8), c = i % (DK / 8);
+            if (i < NCH) *reinterpret_cast<uint4*>(qs + (c / 8) * C::QKB + sw128_offset(r, c % 8)) = v[u];
+          }
         }
         for (int r = lane; r < C::QROWS; r += 32) {
           const int qq = r / HP, h = r % HP;
@@ -169,6 +214,7 @@ __global__ void __launch_bounds__(POOL ? kPoolThreads : kThreads, 1)
         __syncwarp();
         if (lane == 0) mbar_arrive(&qfull[slot]);
         prev_bg = bg;
+        }
       }
       const int stage = static_cast<int>(it % S);
       if (it >= S && !mbar_wait(&empty[stage], ((it / S) - 1) & 1, abort_flag, p.err)) { ok = false; break; }
@@ -181,16 +227,19 @@ __global__ void __launch_bounds__(POOL ? kPoolThreads : kThreads, 1)
           for (int kb = 0; kb < C::KB; ++kb) tma_load_2d(dst + kb * kKBlockBytes, &kmap, &full[stage], kb * 64, row);
         }
       } else {
-        const int64_t qrow = static_cast<int64_t>(b) * p.Q + g;   // NQ == 1 for pools
         {
-          const int r = ptid;                                     // one row per producer thread
-          const int64_t slot_i = static_cast<int64_t>(t) * kTileRows + r;
-          int64_t id = slot_i < L ? p.pool[qrow * p.P + slot_i] : -1;
-          const bool valid = id >= 0 && id < p.N;
-          const uint16_t* src = p.k + (static_cast<int64_t>(b) * p.N + (valid ? id : 0)) * DK;
+          int32_t ids[8];
 #pragma unroll
-          for (int c = 0; c < DK / 8; ++c)
-            cp_async_16(dst + (c / 8) * kKBlockBytes + sw128_offset(r, c % 8), src + c * 8, valid ? 16u : 0u);
+          for (int i = 0; i < 8; ++i) ids[i] = next_ids[i];
+          if (u + 1 < u1) pool_ids(u + 1, next_ids);             // in flight during this unit
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            const bool valid = ids[i] >= 0 && ids[i] < p.N;
+            const uint16_t* src = p.k + (static_cast<int64_t>(b) * p.N + (valid ? ids[i] : 0)) * DK + c16 * 8;
+#pragma unroll
+            for (int kb = 0; kb < C::KB; ++kb)
+              cp_async_16(dst + kb * kKBlockBytes + sw128_offset(rg + 16 * i, c16), src + kb * 64, valid ? 16u : 0u);
+          }
         }
         cp_async_commit();
         // keep kLag stages of copies in flight; stage it-kLag is complete now
@@ -272,6 +321,9 @@ __global__ void __launch_bounds__(POOL ? kPoolThreads : kThreads, 1)
         prev_bg = bg;
       }
       const int acc = static_cast<int>(it & 1);
+      const int64_t e = static_cast<int64_t>(t) * kTileRows + row;   // entry or pool slot
+      // pool: this row's entry id, loaded while the products are computed
+      const int64_t pid = POOL && e < L ? p.pool[(static_cast<int64_t>(b) * p.Q + g) * p.P + e] : -1;
       if (!mbar_wait(&tfull[acc], (it >> 1) & 1, abort_flag, p.err)) break;
       tc_fence_after();
       const float* w = sW + (qi & 1) * C::QROWS;
@@ -297,13 +349,11 @@ __global__ void __launch_bounds__(POOL ? kPoolThreads : kThreads, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&tempty[acc]);
-      const int64_t e = static_cast<int64_t>(t) * kTileRows + row;   // entry or pool slot
       if (e < L) {
         bool valid = true;
         if (POOL) {
-          const int64_t id = p.pool[(static_cast<int64_t>(b) * p.Q + g) * p.P + e];
-          if (id >= p.N || id < -1) raise_dev_error(p.err, DEVERR_BOUNDS);
-          valid = id >= 0 && id < p.N;
+          if (pid >= p.N || pid < -1) raise_dev_error(p.err, DEVERR_BOUNDS);
+          valid = pid >= 0 && pid < p.N;
         }
 #pragma unroll
         for (int qq = 0; qq < NQ; ++qq) {
@@ -335,6 +385,11 @@ csa2_status run_tc(const void* q, const float* w, const void* k, int B, int Q, i
   if (!POOL) {
     CSA2_TRY(make_tensor_map_bf16_2d(&map, k, static_cast<uint64_t>(B) * N, DK, DK * 2, 64, kTileRows));
   }
+  CUtensorMap qmap;
+  memset(&qmap, 0, sizeof(qmap));
+  const bool q_tma = NQ == 1 && H == HP && (reinterpret_cast<uintptr_t>(q) & 15u) == 0;
+  if (q_tma)
+    CSA2_TRY(make_tensor_map_bf16_2d(&qmap, q, static_cast<uint64_t>(B) * Q * H, DK, DK * 2, 64, HP));
   Params p;
   p.q = static_cast<const uint16_t*>(q);
   p.w = w;
@@ -348,6 +403,7 @@ csa2_status run_tc(const void* q, const float* w, const void* k, int B, int Q, i
   p.P = P;
   p.N = N;
   p.relu = act == CSA2_ACT_RELU ? 1 : 0;
+  p.q_tma = q_tma ? 1 : 0;
   p.n_qgroups = (Q + NQ - 1) / NQ;
   const int64_t L = POOL ? P : N;
   p.n_tiles = static_cast<int>((L + kTileRows - 1) / kTileRows);
@@ -361,7 +417,7 @@ csa2_status run_tc(const void* q, const float* w, const void* k, int B, int Q, i
   if (attr_err != cudaSuccess) return fail(CSA2_ERR_CUDA, "index_scores_tc: smem opt-in failed");
   const int64_t grid = std::min<int64_t>(sm_count(), p.n_units);
   begin_launch(stream);
-  kern<<<static_cast<unsigned>(grid), POOL ? kPoolThreads : kThreads, C::BYTES, stream>>>(map, p);
+  kern<<<static_cast<unsigned>(grid), POOL ? kPoolThreads : kThreads, C::BYTES, stream>>>(map, qmap, p);
   note_launch(POOL ? LK_INDEX_POOL : LK_INDEX, 1, stream);
   return check_launch("index_scores_tc");
 }

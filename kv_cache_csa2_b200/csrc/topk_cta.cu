@@ -135,28 +135,36 @@ __global__ void __launch_bounds__(NT, 1) topk_cta_kernel(CtaParams p) {
   uint32_t kmin = 0xffffffffu, kmax = 0u;
   int nsel = 0;
   const bool vec = (reinterpret_cast<uintptr_t>(s) & 15u) == 0;
-  for (int b0 = w_lo; b0 < w_hi; b0 += 128) {
-    const int i = b0 + 4 * lane;
-    if (i >= w_hi) continue;
-    float f[4];
-    if (vec && i + 3 < w_hi) {
-      const float4 v = __ldg(reinterpret_cast<const float4*>(s + i));
-      f[0] = v.x; f[1] = v.y; f[2] = v.z; f[3] = v.w;
-    } else {
+  // four groups of 128 scores per step: each lane has its four loads in flight
+  for (int b0 = w_lo; b0 < w_hi; b0 += 4 * 128) {
+    float f[4][4];
 #pragma unroll
-      for (int u = 0; u < 4; ++u) f[u] = i + u < w_hi ? __ldg(s + i + u) : __int_as_float(0xff800000);
-    }
-    uint32_t k4[4];
+    for (int g = 0; g < 4; ++g) {
+      const int i = b0 + g * 128 + 4 * lane;
+      if (vec && i + 3 < w_hi) {
+        const float4 v = __ldg(reinterpret_cast<const float4*>(s + i));
+        f[g][0] = v.x; f[g][1] = v.y; f[g][2] = v.z; f[g][3] = v.w;
+      } else {
 #pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      k4[u] = score_key(f[u]);
-      if (k4[u]) {
-        kmin = min(kmin, k4[u]);
-        kmax = max(kmax, k4[u]);
-        ++nsel;
+        for (int u = 0; u < 4; ++u) f[g][u] = i + u < w_hi ? __ldg(s + i + u) : __int_as_float(0xff800000);
       }
     }
-    *reinterpret_cast<uint4*>(keys + i) = make_uint4(k4[0], k4[1], k4[2], k4[3]);
+#pragma unroll
+    for (int g = 0; g < 4; ++g) {
+      const int i = b0 + g * 128 + 4 * lane;
+      if (i >= w_lo + p.seg) break;                 // past this warp's part of the buffer
+      uint32_t k4[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        k4[u] = score_key(f[g][u]);
+        if (k4[u]) {
+          kmin = min(kmin, k4[u]);
+          kmax = max(kmax, k4[u]);
+          ++nsel;
+        }
+      }
+      *reinterpret_cast<uint4*>(keys + i) = make_uint4(k4[0], k4[1], k4[2], k4[3]);
+    }
   }
   kmin = __reduce_min_sync(0xffffffffu, kmin);
   kmax = __reduce_max_sync(0xffffffffu, kmax);
@@ -337,32 +345,32 @@ __global__ void __launch_bounds__(NT, 1) topk_cta_kernel(CtaParams p) {
         gt_m |= (valid && (all[t] || kv[u] > T[t])) << u;
         eq_m |= (valid && !all[t] && kv[u] == T[t]) << u;
       }
-      // equal keys of lower lanes (and of this lane's earlier keys) come first
-      int ne = __popc(eq_m), eq_excl = ne;
+      // position order is lane-major: the keys of lower lanes, then this
+      // lane's earlier keys, come first
+      const unsigned lt = (1u << lane) - 1u;
+      unsigned eb[4];
+      int eq_lower = 0, warp_eq = 0;
 #pragma unroll
-      for (int off = 1; off < 32; off <<= 1) {
-        const int y = __shfl_up_sync(0xffffffffu, eq_excl, off);
-        if (lane >= off) eq_excl += y;
+      for (int u = 0; u < 4; ++u) {
+        eb[u] = __ballot_sync(0xffffffffu, (eq_m >> u) & 1);
+        eq_lower += __popc(eb[u] & lt);
+        warp_eq += __popc(eb[u]);
       }
-      eq_excl -= ne;
-      int sel_m = gt_m, rank = run_eq + eq_excl;
+      int sel_m = gt_m, rank = run_eq + eq_lower;
 #pragma unroll
       for (int u = 0; u < 4; ++u)
         if ((eq_m >> u) & 1) {
           if (rank < take[t]) sel_m |= 1 << u;
           ++rank;
         }
-      const int ns = __popc(sel_m);
-      int sel_excl = ns;
+      int sel_lower = 0, warp_sel = 0;
 #pragma unroll
-      for (int off = 1; off < 32; off <<= 1) {
-        const int y = __shfl_up_sync(0xffffffffu, sel_excl, off);
-        if (lane >= off) sel_excl += y;
+      for (int u = 0; u < 4; ++u) {
+        const unsigned sb = __ballot_sync(0xffffffffu, (sel_m >> u) & 1);
+        sel_lower += __popc(sb & lt);
+        warp_sel += __popc(sb);
       }
-      const int warp_sel = __shfl_sync(0xffffffffu, sel_excl, 31);
-      const int warp_eq = __reduce_add_sync(0xffffffffu, ne);
-      sel_excl -= ns;
-      int pos = run_sel + sel_excl;
+      int pos = run_sel + sel_lower;
 #pragma unroll
       for (int u = 0; u < 4; ++u)
         if ((sel_m >> u) & 1) {
