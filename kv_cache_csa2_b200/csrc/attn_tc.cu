@@ -265,8 +265,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         off[i] = static_cast<int64_t>(id >= 0 ? id : 0) * DV;     // empty slot: masked later
       }
-#pragma unroll
-      for (int kb = 0; kb < kKB; ++kb) {
+#pragma unroll 1
+      for (int kb = 0; kb < kKB; ++kb) {          // not unrolled: one short body, re-executed
 #pragma unroll
         for (int i = 0; i < 8; ++i)
           cp_async_16(sKV + kb * kKBBytes + (grow0 + 16 * i) * 128 + swz, base + off[i] + kb * 64, 16);
@@ -428,27 +428,37 @@ __global__ void __launch_bounds__(kThreads, 1)
       // weights of the T partials exp(m_j - M), the query's M and L
       if (p.bulk) {
         ok = mbar_wait(r_full, par, abort_flag, p.err) && ok;
-        if (et < HA) {
-          // T <= 32 here: all loads first, then the max, the weights and L in tile order
-          const uint32_t mlj = smem_u32(sP) + et * 4;  // m_j at + j*512, l_j at + j*512 + 256
-          float mj[32], lj[32];
+        // all 128 threads: head h = et % 64 takes tiles j = half, half + 2, ...
+        // (half = et / 64); every load is issued before any is used
+        {
+          const int h = et & (HA - 1), half = et >> 6;
+          const uint32_t mlj = smem_u32(sP) + h * 4;    // m_j at + j*512, l_j at + j*512 + 256
+          float mj[16], lj[16];                          // T <= 32: at most 16 tiles per half
 #pragma unroll
-          for (int j = 0; j < 32; ++j) {
-            mj[j] = j < p.T ? lds_f32(mlj + j * 2 * HA * 4) : -INFINITY;
-            lj[j] = j < p.T ? lds_f32(mlj + j * 2 * HA * 4 + HA * 4) : 0.0f;
+          for (int i = 0; i < 16; ++i) {
+            const int j = half + 2 * i;
+            mj[i] = j < p.T ? lds_f32(mlj + j * 2 * HA * 4) : -INFINITY;
+            lj[i] = j < p.T ? lds_f32(mlj + j * 2 * HA * 4 + HA * 4) : 0.0f;
           }
-          float M = -INFINITY;
+          float mh = -INFINITY;
 #pragma unroll
-          for (int j = 0; j < 32; ++j) M = fmaxf(M, mj[j]);
-          float L = 0.0f;
+          for (int i = 0; i < 16; ++i) mh = fmaxf(mh, mj[i]);
+          sRed[half * HA + h] = mh;
+          epi_bar();
+          const float M = fmaxf(sRed[h], sRed[HA + h]);
+          float Lh = 0.0f;                               // this half's tiles, in tile order
 #pragma unroll
-          for (int j = 0; j < 32; ++j) {
-            const float wj = rescale(mj[j], M);
-            if (j < p.T) sW[j * HA + et] = wj;
-            L += lj[j] * wj;
+          for (int i = 0; i < 16; ++i) {
+            const float wj = rescale(mj[i], M);
+            if (half + 2 * i < p.T) sW[(half + 2 * i) * HA + h] = wj;
+            Lh += lj[i] * wj;
           }
-          sML2[et] = M;
-          sML2[HA + et] = L;
+          sRed[2 * HA + half * HA + h] = Lh;
+          epi_bar();
+          if (et < HA) {
+            sML2[et] = M;
+            sML2[HA + et] = sRed[2 * HA + et] + sRed[3 * HA + et];   // even tiles, then odd tiles
+          }
         }
       } else {
         float* dstv = et < HA ? sW : sLv;                // m_j into sW, l_j into sLv
@@ -490,7 +500,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int u = 0; u < 4; ++u) acc[u] = make_float4(0.f, 0.f, 0.f, 0.f);
           if (p.bulk) {
-#pragma unroll 4
+#pragma unroll 2
             for (int j = 0; j < p.T; ++j) {
               float4 v[4];
 #pragma unroll

@@ -61,6 +61,7 @@ struct Smem {
   int nsel;                                // selectable keys in the row
   int ncand[kTracks];
   int bin[kTracks], above[kTracks];
+  int eqtot[kTracks];                      // keys equal to the threshold, whole row
 };
 
 // Exclusive block-wide prefix sum (thread order) of one int; *total = sum.
@@ -327,42 +328,58 @@ __global__ void __launch_bounds__(NT, 1) topk_cta_kernel(CtaParams p) {
     const int g_before = gi - g, e_before = ei - e;
     S.off_eq[t][lane] = e_before;
     S.off_sel[t][lane] = g_before + min(e_before, take[t]);
+    if (lane == 31) S.eqtot[t] = ei;
   }
   __syncthreads();
 #pragma unroll
   for (int t = 0; t < kTracks; ++t) {
     if (t >= p.ntracks) break;
     int32_t* o = p.out[t] + r * static_cast<int64_t>(p.count[t]);
-    int run_sel = S.off_sel[t][warp], run_eq = S.off_eq[t][warp];
+    const int sel_start = S.off_sel[t][warp];
+    int run_sel = sel_start, run_eq = S.off_eq[t][warp];
+    // one selection: the warp's picks are compacted in order into its own part
+    // of the key buffer (never past the keys it has read), then copied out
+    // with coalesced stores; two selections: stored directly
+    const bool stage = p.ntracks == 1;
+    // every key equal to T is taken (the usual case): no ranks among equal keys
+    const bool simple = all[t] || take[t] >= S.eqtot[t];
+    const uint32_t thr = all[t] ? 1u : T[t];
+    const unsigned lt = (1u << lane) - 1u;
     for (int b0 = w_lo; b0 < w_hi; b0 += 128) {
       const int i = b0 + 4 * lane;
       const uint4 k4 = *reinterpret_cast<const uint4*>(keys + i);
       const uint32_t kv[4] = {k4.x, k4.y, k4.z, k4.w};
-      int gt_m = 0, eq_m = 0;                  // bit u: key u is above / equal to T
+      int sel_m = 0;                           // bit u: key u is taken
+      int warp_eq = 0;
+      if (simple) {
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const bool valid = kv[u] != 0u && i + u < w_hi;
-        gt_m |= (valid && (all[t] || kv[u] > T[t])) << u;
-        eq_m |= (valid && !all[t] && kv[u] == T[t]) << u;
-      }
-      // position order is lane-major: the keys of lower lanes, then this
-      // lane's earlier keys, come first
-      const unsigned lt = (1u << lane) - 1u;
-      unsigned eb[4];
-      int eq_lower = 0, warp_eq = 0;
+        for (int u = 0; u < 4; ++u) sel_m |= (kv[u] >= thr && i + u < w_hi) << u;
+        if (!__any_sync(0xffffffffu, sel_m)) continue;
+      } else {
+        int eq_m = 0;                          // bit u: key u equals T
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        eb[u] = __ballot_sync(0xffffffffu, (eq_m >> u) & 1);
-        eq_lower += __popc(eb[u] & lt);
-        warp_eq += __popc(eb[u]);
-      }
-      int sel_m = gt_m, rank = run_eq + eq_lower;
-#pragma unroll
-      for (int u = 0; u < 4; ++u)
-        if ((eq_m >> u) & 1) {
-          if (rank < take[t]) sel_m |= 1 << u;
-          ++rank;
+        for (int u = 0; u < 4; ++u) {
+          const bool valid = kv[u] != 0u && i + u < w_hi;
+          sel_m |= (valid && kv[u] > T[t]) << u;
+          eq_m |= (valid && kv[u] == T[t]) << u;
         }
+        // position order is lane-major: the keys of lower lanes, then this
+        // lane's earlier keys, come first
+        int eq_lower = 0;
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const unsigned eb = __ballot_sync(0xffffffffu, (eq_m >> u) & 1);
+          eq_lower += __popc(eb & lt);
+          warp_eq += __popc(eb);
+        }
+        int rank = run_eq + eq_lower;
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+          if ((eq_m >> u) & 1) {
+            if (rank < take[t]) sel_m |= 1 << u;
+            ++rank;
+          }
+      }
       int sel_lower = 0, warp_sel = 0;
 #pragma unroll
       for (int u = 0; u < 4; ++u) {
@@ -374,11 +391,22 @@ __global__ void __launch_bounds__(NT, 1) topk_cta_kernel(CtaParams p) {
 #pragma unroll
       for (int u = 0; u < 4; ++u)
         if ((sel_m >> u) & 1) {
-          if (pos < p.count[t]) o[pos] = p.ids ? p.ids[r * p.L + i + u] : i + u;
+          if (stage)
+            keys[w_lo + (pos - sel_start)] = static_cast<uint32_t>(i + u);
+          else if (pos < p.count[t])
+            o[pos] = p.ids ? p.ids[r * p.L + i + u] : i + u;
           ++pos;
         }
       run_sel += warp_sel;
       run_eq += warp_eq;
+    }
+    if (stage) {
+      __syncwarp();
+      for (int j = lane; j < run_sel - sel_start; j += 32) {
+        const int q = sel_start + j;
+        const int posn = static_cast<int>(keys[w_lo + j]);
+        if (q < p.count[t]) o[q] = p.ids ? p.ids[r * p.L + posn] : posn;
+      }
     }
   }
   // padding: positions beyond the selectable keys

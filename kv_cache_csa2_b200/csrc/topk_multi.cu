@@ -14,7 +14,12 @@
 // histogram into the row's global histogram, the row's CTAs meet at a barrier
 // (a counter in global memory, bounded wait), and every CTA then derives the
 // same next key prefix from the global histogram; a row held by one CTA needs
-// neither.  After the last pass, the threshold key T and the number
+// neither.  When, after the first pass, few keys share each selection's
+// threshold bin (at most kCandCap), the CTAs copy those keys and positions to
+// a per-row candidate list with their counts of keys above the bin, meet once
+// more, and each CTA finishes alone from the list: the remaining digits, its
+// output offset and its share of the keys equal to T.  Otherwise, after the
+// last pass, the threshold key T and the number
 // of keys equal to T to take are known; the CTAs exchange per-chunk counts
 // (one more barrier) and each writes its selected positions, in position
 // order, at the offset the lower chunks leave -- ties at T go to the lowest
@@ -42,6 +47,7 @@ constexpr int kPasses = 3;                 // 32 bits need at most three 12-bit 
 constexpr int kTracks = 2;
 constexpr int kMaxRowsMulti = 1024;
 constexpr int kMaxC = 64;
+constexpr int kCandCap = 4096;            // candidate keys per row and selection
 
 struct SelParams {
   const float* scores;
@@ -54,6 +60,9 @@ struct SelParams {
   int* cnt;           // [rows][C][kTracks][2]
   unsigned* minmax;   // [rows][2]: max of ~key (so the min), max key
   unsigned* bar;      // [rows]
+  uint32_t* ckey;     // [rows][kTracks][kCandCap] keys of the threshold bin after pass 0
+  int32_t* cpos;      // [rows][kTracks][kCandCap] their positions
+  int* ccnt;          // [rows][kTracks]
   int* err;
 };
 
@@ -230,6 +239,7 @@ __global__ void __launch_bounds__(kT) topk_multi_kernel(SelParams p) {
       mask[t] = cmask;
     }
     int lowbit = 32 - common;               // bits [lowbit-1 : 0] still undecided
+    bool use_cand = false;
     for (int pass = 0; pass < kPasses && lowbit > 0 && ok; ++pass) {
       const int width = lowbit >= kDigit ? kDigit : lowbit;
       const int shift = lowbit - width;
@@ -290,6 +300,138 @@ __global__ void __launch_bounds__(kT) topk_multi_kernel(SelParams p) {
         __syncthreads();
       }
       lowbit = shift;
+      if (pass == 0 && C > 1) {
+        // few keys share the threshold bin of every selection: finish on those
+        // candidates instead of more passes over the row (the same decision in
+        // every CTA of the row: it reads the row's histogram)
+        bool fits = true;
+        for (int t = 0; t < p.ntracks; ++t)
+          if (!all[t] && __ldcg(&ghp[t * kBins + sh_bin[t]]) > kCandCap) fits = false;
+        if (fits) {
+          use_cand = true;
+          break;
+        }
+      }
+    }
+    int* cr = p.cnt + r * C * kTracks * 2;
+    if (use_cand && ok) {
+      // (1) candidates: keys of each selection's threshold bin, with their
+      // positions; and this chunk's keys above that bin
+      uint32_t* ck = p.ckey + r * kTracks * kCandCap;
+      int32_t* cp = p.cpos + r * kTracks * kCandCap;
+      int* cc = p.ccnt + r * kTracks;
+      for (int t = 0; t < p.ntracks; ++t) {
+        const uint32_t bin_max = prefix[t] | ~mask[t];
+        int above = 0;
+        for (int i0 = 0; i0 < n; i0 += kT) {
+          const int i = i0 + tid;
+          const uint32_t key = i < n ? keys[i] : 0u;
+          const bool sel = key != 0u && (all[t] || key > bin_max);
+          const bool in_bin = key != 0u && !all[t] && (key & mask[t]) == prefix[t];
+          above += sel ? 1 : 0;
+          const unsigned bal = __ballot_sync(0xffffffffu, in_bin);
+          int base = 0;
+          if (lane == 0 && bal) base = atomicAdd(&cc[t], __popc(bal));
+          base = __shfl_sync(0xffffffffu, base, 0);
+          if (in_bin) {
+            const int idx = base + __popc(bal & ((1u << lane) - 1u));
+            ck[t * kCandCap + idx] = key;
+            cp[t * kCandCap + idx] = static_cast<int32_t>(lo + i);
+          }
+        }
+        int tot;
+        block_scan(above, ws, &tot);
+        if (tid == 0) cr[(c * kTracks + t) * 2] = tot;
+      }
+      ok = row_barrier(ctr, C * (++epoch), p.err, &abort_s);
+      // (2) every CTA refines the threshold over the candidates (same result)
+      for (int t = 0; t < p.ntracks && ok; ++t) {
+        if (all[t]) continue;
+        const int nc = __ldcg(&cc[t]);
+        int lb = lowbit;
+        while (lb > 0) {
+          const int width = lb >= kDigit ? kDigit : lb;
+          const int shift = lb - width;
+          const int bins = 1 << width;
+          for (int i = tid; i < kBins; i += kT) hist_s[t][i] = 0;
+          __syncthreads();
+          for (int i = tid; i < nc; i += kT) {
+            const uint32_t key = __ldcg(&ck[t * kCandCap + i]);
+            if ((key & mask[t]) == prefix[t]) atomicAdd(&hist_s[t][(key >> shift) & (bins - 1)], 1);
+          }
+          __syncthreads();
+          const int per = (bins + kT - 1) / kT;
+          int h[kBins / kT];
+          int local = 0;
+#pragma unroll
+          for (int u = 0; u < kBins / kT; ++u) {
+            const int bin = tid * per + u;
+            h[u] = (u < per && bin < bins) ? hist_s[t][bin] : 0;
+            local += h[u];
+          }
+          int total;
+          const int before = block_scan(local, ws, &total);
+          int ab = total - before - local;
+#pragma unroll
+          for (int u = kBins / kT - 1; u >= 0; --u) {
+            if (u < per && ab < kk[t] && ab + h[u] >= kk[t]) {
+              sh_bin[t] = tid * per + u;
+              sh_above[t] = ab;
+            }
+            ab += h[u];
+          }
+          __syncthreads();
+          prefix[t] |= static_cast<uint32_t>(sh_bin[t]) << shift;
+          mask[t] |= static_cast<uint32_t>(bins - 1) << shift;
+          kk[t] -= sh_above[t];
+          __syncthreads();
+          lb = shift;
+        }
+        // (3) this chunk's offset and its share of the keys equal to T: from
+        // the lower chunks' counts above the bin and the candidates' positions
+        const uint32_t Tt = prefix[t];
+        int gt_b = 0, eq_b = 0, eq_in = 0;
+        for (int i = tid; i < nc; i += kT) {
+          const uint32_t key = __ldcg(&ck[t * kCandCap + i]);
+          const int64_t pos = __ldcg(&cp[t * kCandCap + i]);
+          if (pos < lo) {
+            gt_b += key > Tt ? 1 : 0;
+            eq_b += key == Tt ? 1 : 0;
+          } else if (pos < lo + n) {
+            eq_in += key == Tt ? 1 : 0;
+          }
+        }
+        for (int cc2 = tid; cc2 < c; cc2 += kT) gt_b += __ldcg(&cr[(cc2 * kTracks + t) * 2]);
+        int tg, te, ti;
+        block_scan(gt_b, ws, &tg);
+        block_scan(eq_b, ws, &te);
+        block_scan(eq_in, ws, &ti);
+        if (tid == 0) {
+          sh_off[t] = tg + min(te, kk[t]);
+          sh_take[t] = max(0, min(kk[t] - te, ti));
+          sh_all_sel[t] = p.count[t];
+        }
+      }
+      if (ok) {
+        for (int t = 0; t < p.ntracks; ++t) {
+          if (!all[t]) continue;          // every selectable key: offsets from the counts alone
+          int before = 0, tot_all = 0;
+          for (int cc2 = tid; cc2 < C; cc2 += kT) {
+            const int v = __ldcg(&cr[(cc2 * kTracks + t) * 2]);
+            if (cc2 < c) before += v;
+            tot_all += v;
+          }
+          int tb, ta;
+          block_scan(before, ws, &tb);
+          block_scan(tot_all, ws, &ta);
+          if (tid == 0) {
+            sh_off[t] = tb;
+            sh_take[t] = 0;
+            sh_all_sel[t] = ta;
+          }
+        }
+      }
+      __syncthreads();
     }
     if (common >= 32 && ok) {               // every selectable key is the same value
 #pragma unroll
@@ -323,8 +465,7 @@ __global__ void __launch_bounds__(kT) topk_multi_kernel(SelParams p) {
       }
     }
     __syncthreads();
-    int* cr = p.cnt + r * C * kTracks * 2;
-    if (tid < kTracks) {
+    if (!use_cand && tid < kTracks) {
       int g = 0, e = 0;
       for (int w = 0; w < kT / 32; ++w) {
         g += seg_gt[tid][w];
@@ -333,9 +474,9 @@ __global__ void __launch_bounds__(kT) topk_multi_kernel(SelParams p) {
       cr[(c * kTracks + tid) * 2] = g;
       cr[(c * kTracks + tid) * 2 + 1] = e;
     }
-    if (ok && C > 1) ok = row_barrier(ctr, C * (++epoch), p.err, &abort_s);
+    if (ok && C > 1 && !use_cand) ok = row_barrier(ctr, C * (++epoch), p.err, &abort_s);
     __syncthreads();
-    if (tid < p.ntracks && ok) {
+    if (tid < p.ntracks && ok && !use_cand) {
       int off = 0, eq_left = need_eq[tid], take = 0, all_sel = 0;
       for (int cc = 0; cc < C; ++cc) {
         const int g = __ldcg(&cr[(cc * kTracks + tid) * 2]);
@@ -429,9 +570,16 @@ bool multi_applies(int64_t rows, int64_t L) {
   return C <= kMaxC;
 }
 
-size_t ws_bytes_for(int64_t rows, int64_t L) {
+// Workspace: [hist | cnt | minmax | bar | ccnt] (cleared before each launch),
+// then the candidate lists [ckey | cpos] (written before being read).
+size_t ws_cleared_bytes(int64_t rows, int64_t L) {
   const int64_t C = (L + chunk_for(L) - 1) / chunk_for(L);
-  return static_cast<size_t>(rows) * (kPasses * kTracks * kBins + C * kTracks * 2 + 2 + 1) * 4 + 256;
+  const size_t words = static_cast<size_t>(rows) * (kPasses * kTracks * kBins + C * kTracks * 2 + 2 + 1 + kTracks);
+  return (words * 4 + 255) & ~size_t(255);
+}
+
+size_t ws_bytes_for(int64_t rows, int64_t L) {
+  return ws_cleared_bytes(rows, L) + static_cast<size_t>(rows) * kTracks * kCandCap * 8 + 256;
 }
 
 }  // namespace
@@ -470,10 +618,14 @@ csa2_status launch_select_topk2(const float* scores, int64_t rows, int64_t L, in
   p.cnt = p.hist + rows * kPasses * kTracks * kBins;
   p.minmax = reinterpret_cast<unsigned*>(p.cnt + rows * C * kTracks * 2);
   p.bar = p.minmax + rows * 2;
+  p.ccnt = reinterpret_cast<int*>(p.bar + rows);
+  const size_t cleared = ws_cleared_bytes(rows, L);
+  p.ckey = reinterpret_cast<uint32_t*>(static_cast<char*>(ws) + cleared);
+  p.cpos = reinterpret_cast<int32_t*>(p.ckey + rows * kTracks * kCandCap);
   p.err = device_error_word();
-  if (C > 1) {          // row histograms, counts and barrier counters start at zero
+  if (C > 1) {          // row histograms, counts, barrier and candidate counters start at zero
     begin_launch(stream);
-    if (cudaMemsetAsync(ws, 0, need, stream) != cudaSuccess) return check_launch("select_topk: clear");
+    if (cudaMemsetAsync(ws, 0, cleared, stream) != cudaSuccess) return check_launch("select_topk: clear");
     note_launch(LK_OTHER, 1, stream);
   }
   void* args[] = {&p};
