@@ -106,6 +106,13 @@ __device__ __forceinline__ void warp_transpose_reduce(float (&v)[64], int lane) 
     }
   }
 }
+// Max of one float over the 32 lanes of a warp (every lane gets it).
+__device__ __forceinline__ float warp_max_f32(float v) {
+  float r;
+  asm volatile("redux.sync.max.f32 %0, %1, 0xffffffff;" : "=f"(r) : "f"(v));
+  return r;
+}
+
 __device__ __forceinline__ int reduced_head_base(int lane) {
   return ((lane >> 4) & 1) * 32 + ((lane >> 3) & 1) * 16 + ((lane >> 2) & 1) * 8 +
          ((lane >> 1) & 1) * 4 + (lane & 1) * 2;
@@ -298,26 +305,24 @@ __global__ void __launch_bounds__(kThreads, 1)
       float x[HA];
       if (ok) {
         tc_fence_after();
-        uint32_t v[32];
+        uint32_t v0[32], v1[32];
+        tmem_ld32(tmem + lane_off + S_COL, v0);
+        tmem_ld32(tmem + lane_off + S_COL + 32, v1);
+        tmem_wait_ld();
 #pragma unroll
-        for (int half = 0; half < 2; ++half) {
-          tmem_ld32(tmem + lane_off + S_COL + 32 * half, v);
-          tmem_wait_ld();
-#pragma unroll
-          for (int h = 0; h < 32; ++h) x[32 * half + h] = valid ? p.scale * __uint_as_float(v[h]) : -INFINITY;
+        for (int h = 0; h < 32; ++h) {
+          x[h] = valid ? p.scale * __uint_as_float(v0[h]) : -INFINITY;
+          x[32 + h] = valid ? p.scale * __uint_as_float(v1[h]) : -INFINITY;
         }
       } else {
 #pragma unroll
         for (int h = 0; h < HA; ++h) x[h] = -INFINITY;
       }
-      // the tile's per-head max m
-      {
-        float red[HA];
+      // the tile's per-head max m: one warp-wide max per head, then over the 4 warps
 #pragma unroll
-        for (int h = 0; h < HA; ++h) red[h] = x[h];
-        warp_transpose_reduce<true>(red, lane);
-        sRed[ew * HA + hb] = red[0];
-        sRed[ew * HA + hb + 1] = red[1];
+      for (int h = 0; h < HA; ++h) {
+        const float mh = warp_max_f32(x[h]);
+        if (lane == 0) sRed[ew * HA + h] = mh;
       }
       epi_bar();
       if (et < HA)
@@ -371,14 +376,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int dim = mc * 128 + row;
         const uint32_t srow = kv0 + dim * (HA * 4);
         if (ok) {
+          uint32_t v0[32], v1[32];
+          tmem_ld32(tmem + lane_off + O_COL + 64 * mc, v0);
+          tmem_ld32(tmem + lane_off + O_COL + 64 * mc + 32, v1);
+          tmem_wait_ld();
 #pragma unroll
-          for (int half = 0; half < 2; ++half) {
-            uint32_t v[32];
-            tmem_ld32(tmem + lane_off + O_COL + 64 * mc + 32 * half, v);
-            tmem_wait_ld();
-#pragma unroll
-            for (int c = 0; c < 8; ++c)
-              sts_v4u(srow + (((8 * half + c) ^ (dim & 7)) << 4), v[4 * c], v[4 * c + 1], v[4 * c + 2], v[4 * c + 3]);
+          for (int c = 0; c < 8; ++c) {
+            sts_v4u(srow + ((c ^ (dim & 7)) << 4), v0[4 * c], v0[4 * c + 1], v0[4 * c + 2], v0[4 * c + 3]);
+            sts_v4u(srow + (((8 + c) ^ (dim & 7)) << 4), v1[4 * c], v1[4 * c + 1], v1[4 * c + 2], v1[4 * c + 3]);
           }
         }
         fence_proxy_async_smem();

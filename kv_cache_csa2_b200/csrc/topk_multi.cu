@@ -28,7 +28,8 @@
 //
 // The launch is cooperative (all CTAs resident); CTA groups loop over rows,
 // each row having its own counter, histogram and count slots in the
-// workspace, which is cleared before the launch.
+// workspace; the counters and ranges are cleared before the launch, the
+// histograms by the kernel itself.
 #include <algorithm>
 #include <cstdlib>
 #include <mutex>
@@ -56,10 +57,10 @@ struct SelParams {
   int count[kTracks];
   const int32_t* ids;
   int32_t* out[kTracks];
-  int* hist;          // [rows][kPasses][kTracks][kBins]
+  int* hist;          // [rows][kPasses][kTracks][kBins], cleared by the kernel
   int* cnt;           // [rows][C][kTracks][2]
-  unsigned* minmax;   // [rows][2]: max of ~key (so the min), max key
-  unsigned* bar;      // [rows]
+  unsigned* minmax;   // [rows][2]: max of ~key (so the min), max key; zero at launch
+  unsigned* bar;      // [rows], zero at launch
   uint32_t* ckey;     // [rows][kTracks][kCandCap] keys of the threshold bin after pass 0
   int32_t* cpos;      // [rows][kTracks][kCandCap] their positions
   int* ccnt;          // [rows][kTracks]
@@ -215,6 +216,14 @@ __global__ void __launch_bounds__(kT) topk_multi_kernel(SelParams p) {
     }
     __syncthreads();
     if (C > 1) {      // the row's range over all chunks
+      // this CTA's share of the row's histograms (and, for chunk 0, the
+      // candidate counters) start at zero; the barrier below publishes it
+      {
+        const int words = kPasses * kTracks * kBins;
+        const int per = (words + C - 1) / C;
+        for (int i = c * per + tid; i < min(words, (c + 1) * per); i += kT) gh[i] = 0;
+        if (c == 0 && tid < kTracks) p.ccnt[r * kTracks + tid] = 0;
+      }
       if (tid == 0) {
         atomicMax(&gmm[0], ~sh_min);
         atomicMax(&gmm[1], sh_max);
@@ -570,16 +579,18 @@ bool multi_applies(int64_t rows, int64_t L) {
   return C <= kMaxC;
 }
 
-// Workspace: [hist | cnt | minmax | bar | ccnt] (cleared before each launch),
-// then the candidate lists [ckey | cpos] (written before being read).
-size_t ws_cleared_bytes(int64_t rows, int64_t L) {
-  const int64_t C = (L + chunk_for(L) - 1) / chunk_for(L);
-  const size_t words = static_cast<size_t>(rows) * (kPasses * kTracks * kBins + C * kTracks * 2 + 2 + 1 + kTracks);
-  return (words * 4 + 255) & ~size_t(255);
+// Workspace: [minmax | bar] (cleared before each launch), then [hist | ccnt]
+// (cleared by the kernel itself before its first barrier), [cnt] and the
+// candidate lists [ckey | cpos] (written before being read).
+size_t ws_cleared_bytes(int64_t rows) {
+  return (static_cast<size_t>(rows) * 3 * 4 + 255) & ~size_t(255);
 }
 
 size_t ws_bytes_for(int64_t rows, int64_t L) {
-  return ws_cleared_bytes(rows, L) + static_cast<size_t>(rows) * kTracks * kCandCap * 8 + 256;
+  const int64_t C = (L + chunk_for(L) - 1) / chunk_for(L);
+  const size_t words = static_cast<size_t>(rows) * (kPasses * kTracks * kBins + kTracks + C * kTracks * 2);
+  return ws_cleared_bytes(rows) + ((words * 4 + 255) & ~size_t(255)) +
+         static_cast<size_t>(rows) * kTracks * kCandCap * 8 + 256;
 }
 
 }  // namespace
@@ -614,16 +625,17 @@ csa2_status launch_select_topk2(const float* scores, int64_t rows, int64_t L, in
   p.ids = ids;
   p.out[0] = out0;
   p.out[1] = out1;
-  p.hist = static_cast<int*>(ws);
-  p.cnt = p.hist + rows * kPasses * kTracks * kBins;
-  p.minmax = reinterpret_cast<unsigned*>(p.cnt + rows * C * kTracks * 2);
+  const size_t cleared = ws_cleared_bytes(rows);
+  p.minmax = static_cast<unsigned*>(ws);
   p.bar = p.minmax + rows * 2;
-  p.ccnt = reinterpret_cast<int*>(p.bar + rows);
-  const size_t cleared = ws_cleared_bytes(rows, L);
-  p.ckey = reinterpret_cast<uint32_t*>(static_cast<char*>(ws) + cleared);
+  p.hist = reinterpret_cast<int*>(static_cast<char*>(ws) + cleared);
+  p.ccnt = p.hist + rows * kPasses * kTracks * kBins;
+  p.cnt = p.ccnt + rows * kTracks;
+  const size_t words = static_cast<size_t>(rows) * (kPasses * kTracks * kBins + kTracks + C * kTracks * 2);
+  p.ckey = reinterpret_cast<uint32_t*>(static_cast<char*>(ws) + cleared + ((words * 4 + 255) & ~size_t(255)));
   p.cpos = reinterpret_cast<int32_t*>(p.ckey + rows * kTracks * kCandCap);
   p.err = device_error_word();
-  if (C > 1) {          // row histograms, counts, barrier and candidate counters start at zero
+  if (C > 1) {          // row ranges and barrier counters start at zero
     begin_launch(stream);
     if (cudaMemsetAsync(ws, 0, cleared, stream) != cudaSuccess) return check_launch("select_topk: clear");
     note_launch(LK_OTHER, 1, stream);
