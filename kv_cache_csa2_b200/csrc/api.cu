@@ -139,6 +139,11 @@ int* device_error_word() {
   return g_err_ptr[dev];
 }
 
+bool pdl_enabled() {
+  static const bool on = getenv("CSA2_NO_PDL") == nullptr;
+  return on;
+}
+
 int sm_count() {
   const int dev = current_device();
   std::lock_guard<std::mutex> lk(g_dev_mu);
@@ -390,12 +395,15 @@ csa2_status csa2_index_topk(csa2_mode mode, const void* q, const float* w, const
   const size_t sbytes = align256(static_cast<size_t>(rows) * L * sizeof(float));
   void* sel_ws = static_cast<char*>(workspace) + sbytes;
   const size_t sel_bytes = workspace_bytes - sbytes;
+  // the dual selection's counters are cleared first, so that it follows the
+  // scoring kernel directly (programmatic dependent launch)
+  if (pool_out) CSA2_TRY(select_topk_clear(rows, L, sel_ws, sel_bytes, s));
   CSA2_TRY(launch_index_scores(q, w, k, B, Q, H, d, N, n_visible, pool_in, pool_in ? P_in : 0, act,
                                scores, s));
   if (pool_out) {
     // the pool and the top-k in the same selection passes when the kernel applies
     const csa2_status st = launch_select_topk2(scores, rows, L, k_top, nullptr, topk_out, P_out,
-                                               pool_out, sel_ws, sel_bytes, s);
+                                               pool_out, sel_ws, sel_bytes, s, true);
     if (st != CSA2_ERR_UNSUPPORTED) return st;
   }
   CSA2_TRY(launch_select_topk(scores, rows, L, k_top, pool_in, topk_out, sel_ws, sel_bytes, s));

@@ -188,6 +188,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  pdl_wait();                                  // the selection comes from the kernel before
 
   if (warp == 0) {
     // ------------------------------------------------------------ q loader
@@ -698,11 +699,12 @@ csa2_status launch_sparse_attn_tc(const void* q, const csa2_kv& kv, const int32_
   cfg.blockDim = dim3(kThreads);
   cfg.dynamicSmemBytes = SMEM_BYTES;
   cfg.stream = stream;
-  cudaLaunchAttribute at[1];
+  cudaLaunchAttribute at[2];
   at[0].id = cudaLaunchAttributeCooperative;
   at[0].val.cooperative = 1;
+  at[1] = pdl_attribute();
   cfg.attrs = at;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = 2;
   begin_launch(stream);
   const cudaError_t e = cudaLaunchKernelEx(&cfg, attn_tc_kernel, qmap, p);
   note_launch(LK_ATTN, 1, stream);

@@ -42,6 +42,22 @@ int sm_count();
 
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+// Programmatic dependent launch.  A kernel launched with the attribute from
+// pdl_attribute() may start while the kernel before it on the stream is still
+// running, once every CTA of that kernel has called pdl_release() (or
+// exited); it calls pdl_wait() before it reads anything that kernel wrote
+// (the wait returns when that kernel has completed and its writes are
+// visible).  Disabled when CSA2_NO_PDL is set.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_release() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+bool pdl_enabled();
+inline cudaLaunchAttribute pdl_attribute() {
+  cudaLaunchAttribute a;
+  a.id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  a.val.programmaticStreamSerializationAllowed = pdl_enabled() ? 1 : 0;
+  return a;
+}
+
 #define CSA2_TRY(expr)                          \
   do {                                          \
     csa2_status _s = (expr);                    \

@@ -103,6 +103,7 @@ __global__ void __launch_bounds__(POOL ? kPoolThreads : kThreads, 1)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t L = POOL ? p.P : p.N;
+  pdl_release();                               // the selection kernel may start launching
 
   // balanced contiguous range of units for this CTA
   const int64_t u0 = p.n_units * blockIdx.x / gridDim.x;

@@ -18,9 +18,15 @@ csa2_status launch_index_scores(const void* q, const float* w, const void* k, in
 size_t select_topk_workspace(int64_t rows, int64_t L, int count);
 // Two selections of the same rows in one pass set (multi-CTA kernel); returns
 // CSA2_ERR_UNSUPPORTED when that kernel does not apply to the shape.
+// ws_cleared: select_topk_clear() already ran on this workspace on `stream`
+// (lets the caller clear it before the kernel that writes the scores, so the
+// selection follows that kernel directly).
 csa2_status launch_select_topk2(const float* scores, int64_t rows, int64_t L, int count0,
                                 const int32_t* ids, int32_t* out0, int count1, int32_t* out1,
-                                void* ws, size_t ws_bytes, cudaStream_t stream);
+                                void* ws, size_t ws_bytes, cudaStream_t stream,
+                                bool ws_cleared = false);
+csa2_status select_topk_clear(int64_t rows, int64_t L, void* ws, size_t ws_bytes,
+                              cudaStream_t stream);
 // One CTA per row, no workspace: rows of up to kSelectCtaMaxL scores.
 constexpr int64_t kSelectCtaMaxL = 32768;
 bool select_topk_cta_applies(int64_t rows, int64_t L);

@@ -123,6 +123,8 @@ __global__ void __launch_bounds__(NT, 1) topk_cta_kernel(CtaParams p) {
   const int L = static_cast<int>(p.L);
   const float* s = p.scores + r * p.L;
   const int w_lo = warp * p.seg, w_hi = min(L, w_lo + p.seg);
+  pdl_wait();                                // the scores come from the kernel before
+  pdl_release();
 
   if (tid == 0) {
     S.kmin = 0xffffffffu;
@@ -454,9 +456,21 @@ csa2_status launch_select_topk_cta(const float* scores, int64_t rows, int64_t L,
                                 static_cast<int>(smem_bytes(kSelectCtaMaxL, kSelectCtaMaxL / NW)));
   });
   if (attr != cudaSuccess) return fail(CSA2_ERR_CUDA, "select_topk_cta: shared-memory opt-in failed");
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(rows));
+  cfg.blockDim = dim3(NT);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute at[1] = {pdl_attribute()};
+  cfg.attrs = at;
+  cfg.numAttrs = 1;
   begin_launch(stream);
-  topk_cta_kernel<<<static_cast<unsigned>(rows), NT, smem, stream>>>(p);
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, topk_cta_kernel, p);
   note_launch(LK_TOPK, 1, stream);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return fail(CSA2_ERR_CUDA, "select_topk_cta: launch failed: %s", cudaGetErrorString(e));
+  }
   return check_launch("select_topk_cta");
 }
 

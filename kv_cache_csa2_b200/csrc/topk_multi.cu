@@ -140,6 +140,8 @@ __global__ void __launch_bounds__(kT) topk_multi_kernel(SelParams p) {
   const int c = blockIdx.x % C;
   const int64_t groups = gridDim.x / C;
   if (tid == 0) abort_s = 0;
+  pdl_wait();                               // the scores come from the kernel before
+  pdl_release();
   __syncthreads();
 
   for (int64_t r = blockIdx.x / C; r < p.rows; r += groups) {
@@ -602,7 +604,7 @@ size_t select_topk_multi_workspace(int64_t rows, int64_t L, int) {
 // Up to two selections of the same rows (count1 may be 0 for one).
 csa2_status launch_select_topk2(const float* scores, int64_t rows, int64_t L, int count0,
                                 const int32_t* ids, int32_t* out0, int count1, int32_t* out1,
-                                void* ws, size_t ws_bytes, cudaStream_t stream) {
+                                void* ws, size_t ws_bytes, cudaStream_t stream, bool ws_cleared) {
   if (cta_kernel_takes(rows, L))
     return launch_select_topk_cta(scores, rows, L, count0, ids, out0, count1, out1, stream);
   if (!multi_applies(rows, L)) return CSA2_ERR_UNSUPPORTED;
@@ -635,22 +637,43 @@ csa2_status launch_select_topk2(const float* scores, int64_t rows, int64_t L, in
   p.ckey = reinterpret_cast<uint32_t*>(static_cast<char*>(ws) + cleared + ((words * 4 + 255) & ~size_t(255)));
   p.cpos = reinterpret_cast<int32_t*>(p.ckey + rows * kTracks * kCandCap);
   p.err = device_error_word();
-  if (C > 1) {          // row ranges and barrier counters start at zero
+  if (C > 1 && !ws_cleared) {          // row ranges and barrier counters start at zero
     begin_launch(stream);
     if (cudaMemsetAsync(ws, 0, cleared, stream) != cudaSuccess) return check_launch("select_topk: clear");
     note_launch(LK_OTHER, 1, stream);
   }
-  void* args[] = {&p};
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(groups * C));
+  cfg.blockDim = dim3(kT);
+  cfg.dynamicSmemBytes = static_cast<size_t>(chunk) * 4;
+  cfg.stream = stream;
+  cudaLaunchAttribute at[2];
+  at[0].id = cudaLaunchAttributeCooperative;
+  at[0].val.cooperative = 1;
+  at[1] = pdl_attribute();
+  cfg.attrs = at;
+  cfg.numAttrs = 2;
   begin_launch(stream);
-  const cudaError_t e = cudaLaunchCooperativeKernel(
-      reinterpret_cast<const void*>(topk_multi_kernel), dim3(static_cast<unsigned>(groups * C)),
-      dim3(kT), args, static_cast<size_t>(chunk) * 4, stream);
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, topk_multi_kernel, p);
   note_launch(LK_TOPK, 1, stream);
   if (e != cudaSuccess) {
     cudaGetLastError();
     return fail(CSA2_ERR_CUDA, "select_topk: cooperative launch failed: %s", cudaGetErrorString(e));
   }
   return check_launch("select_topk_multi");
+}
+
+csa2_status select_topk_clear(int64_t rows, int64_t L, void* ws, size_t ws_bytes,
+                              cudaStream_t stream) {
+  if (cta_kernel_takes(rows, L) || !multi_applies(rows, L) || !ws || ws_bytes < ws_bytes_for(rows, L))
+    return CSA2_OK;
+  const int64_t C = (L + chunk_for(L) - 1) / chunk_for(L);
+  if (C <= 1) return CSA2_OK;
+  begin_launch(stream);
+  if (cudaMemsetAsync(ws, 0, ws_cleared_bytes(rows), stream) != cudaSuccess)
+    return check_launch("select_topk: clear");
+  note_launch(LK_OTHER, 1, stream);
+  return CSA2_OK;
 }
 
 csa2_status launch_select_topk_multi(const float* scores, int64_t rows, int64_t L, int count,
