@@ -78,6 +78,8 @@ struct Cfg {
   static constexpr int BYTES = OFF_MISC + 16 + 1024;       // + alignment slack
   static_assert(NCOL % 16 == 0 && NCOL <= 256, "MMA N");
   static_assert(QKB % 1024 == 0 && TILE_A % 1024 == 0, "swizzle atoms must stay 1 KiB aligned");
+  static_assert(BYTES <= 232448, "shared memory");
+  static_assert(!POOL || kLag < STAGES, "pool gathers keep fewer stages in flight than the ring holds");
 };
 
 template <int DK, int NQ, int HP, bool POOL>

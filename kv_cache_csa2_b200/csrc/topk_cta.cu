@@ -61,7 +61,6 @@ struct Smem {
   int nsel;                                // selectable keys in the row
   int ncand[kTracks];
   int bin[kTracks], above[kTracks];
-  int eqtot[kTracks];                      // keys equal to the threshold, whole row
 };
 
 // Exclusive block-wide prefix sum (thread order) of one int; *total = sum.
@@ -184,6 +183,7 @@ __global__ void __launch_bounds__(NT, 1) topk_cta_kernel(CtaParams p) {
   // ---- per track: threshold key T[t], and how many keys equal to T[t] to take
   uint32_t T[kTracks] = {0u, 0u};
   int take[kTracks] = {0, 0};
+  int eqcnt[kTracks] = {0, 0};             // keys equal to T[t] in the row
   bool all[kTracks] = {true, true};        // every selectable key is chosen
   int kk[kTracks];
   uint32_t prefix[kTracks], mask[kTracks];
@@ -204,7 +204,7 @@ __global__ void __launch_bounds__(NT, 1) topk_cta_kernel(CtaParams p) {
   int lowbit = 32 - common;                // key bits [lowbit-1 : 0] still undecided
   if (any && lowbit == 0) {                // one distinct key, more of it than wanted
 #pragma unroll
-    for (int t = 0; t < kTracks; ++t) T[t] = rmin, take[t] = kk[t];
+    for (int t = 0; t < kTracks; ++t) T[t] = rmin, take[t] = kk[t], eqcnt[t] = total_sel;
   } else if (any) {
     // pass 0 over the whole row (one histogram serves both tracks)
     int width = lowbit >= kDigit ? kDigit : lowbit;
@@ -229,6 +229,7 @@ __global__ void __launch_bounds__(NT, 1) topk_cta_kernel(CtaParams p) {
       mask[t] |= ((1u << width) - 1) << shift;
       kk[t] -= S.above[t];
       in_cand[t] = S.hist[0][b] <= kMaxCand;
+      eqcnt[t] = S.hist[0][b];
     }
     __syncthreads();
     if (tid < kTracks) S.ncand[tid] = 0;
@@ -283,6 +284,7 @@ __global__ void __launch_bounds__(NT, 1) topk_cta_kernel(CtaParams p) {
         prefix[t] |= static_cast<uint32_t>(S.bin[t]) << shift;
         mask[t] |= ((1u << width) - 1) << shift;
         kk[t] -= S.above[t];
+        eqcnt[t] = S.hist[t][S.bin[t]];
       }
       __syncthreads();
       lowbit = shift;
@@ -291,24 +293,55 @@ __global__ void __launch_bounds__(NT, 1) topk_cta_kernel(CtaParams p) {
     for (int t = 0; t < kTracks; ++t) T[t] = prefix[t], take[t] = kk[t];
   }
 
-  // ---- ordered write: per-warp counts, offsets over the warps, then positions
+  // ---- ordered write.  One selection whose keys equal to T are all taken (the
+  // usual case): one sweep compacts each warp's picks, in order, into its own
+  // part of the key buffer (never past the keys it has read), then offsets
+  // over the warps and coalesced copies.  Otherwise: per-warp counts of keys
+  // above / equal to T, offsets, and a sweep that ranks the equal keys.
 #pragma unroll
   for (int t = 0; t < kTracks; ++t) {
     if (t >= p.ntracks) break;
+    const bool simple = p.ntracks == 1 && (all[t] || take[t] >= eqcnt[t]);
+    const uint32_t thr = all[t] ? 1u : T[t];
     int g = 0, e = 0;
-    for (int b0 = w_lo; b0 < w_hi; b0 += 128) {
-      const int i = b0 + 4 * lane;
-      const uint4 k4 = *reinterpret_cast<const uint4*>(keys + i);
-      const uint32_t kv[4] = {k4.x, k4.y, k4.z, k4.w};
+    if (simple) {
+      const unsigned lt = (1u << lane) - 1u;
+      for (int b0 = w_lo; b0 < w_hi; b0 += 128) {
+        const int i = b0 + 4 * lane;
+        const uint4 k4 = *reinterpret_cast<const uint4*>(keys + i);
+        const uint32_t kv[4] = {k4.x, k4.y, k4.z, k4.w};
+        int sel_m = 0;
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const bool valid = kv[u] != 0u && i + u < w_hi;
-        g += (valid && (all[t] || kv[u] > T[t])) ? 1 : 0;
-        e += (valid && !all[t] && kv[u] == T[t]) ? 1 : 0;
+        for (int u = 0; u < 4; ++u) sel_m |= (kv[u] >= thr && i + u < w_hi) << u;
+        if (!__any_sync(0xffffffffu, sel_m)) continue;
+        int lower = 0, total = 0;
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const unsigned sb = __ballot_sync(0xffffffffu, (sel_m >> u) & 1);
+          lower += __popc(sb & lt);
+          total += __popc(sb);
+        }
+        int q = g + lower;
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+          if ((sel_m >> u) & 1) keys[w_lo + q++] = static_cast<uint32_t>(i + u);
+        g += total;
       }
+    } else {
+      for (int b0 = w_lo; b0 < w_hi; b0 += 128) {
+        const int i = b0 + 4 * lane;
+        const uint4 k4 = *reinterpret_cast<const uint4*>(keys + i);
+        const uint32_t kv[4] = {k4.x, k4.y, k4.z, k4.w};
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const bool valid = kv[u] != 0u && i + u < w_hi;
+          g += (valid && (all[t] || kv[u] > T[t])) ? 1 : 0;
+          e += (valid && !all[t] && kv[u] == T[t]) ? 1 : 0;
+        }
+      }
+      g = __reduce_add_sync(0xffffffffu, g);
+      e = __reduce_add_sync(0xffffffffu, e);
     }
-    g = __reduce_add_sync(0xffffffffu, g);
-    e = __reduce_add_sync(0xffffffffu, e);
     if (lane == 0) {
       S.seg_gt[t][warp] = g;
       S.seg_eq[t][warp] = e;
@@ -330,7 +363,6 @@ __global__ void __launch_bounds__(NT, 1) topk_cta_kernel(CtaParams p) {
     const int g_before = gi - g, e_before = ei - e;
     S.off_eq[t][lane] = e_before;
     S.off_sel[t][lane] = g_before + min(e_before, take[t]);
-    if (lane == 31) S.eqtot[t] = ei;
   }
   __syncthreads();
 #pragma unroll
@@ -338,50 +370,44 @@ __global__ void __launch_bounds__(NT, 1) topk_cta_kernel(CtaParams p) {
     if (t >= p.ntracks) break;
     int32_t* o = p.out[t] + r * static_cast<int64_t>(p.count[t]);
     const int sel_start = S.off_sel[t][warp];
+    const bool simple = p.ntracks == 1 && (all[t] || take[t] >= eqcnt[t]);
+    if (simple) {
+      for (int j = lane; j < S.seg_gt[t][warp]; j += 32) {
+        const int q = sel_start + j;
+        const int posn = static_cast<int>(keys[w_lo + j]);
+        if (q < p.count[t]) o[q] = p.ids ? p.ids[r * p.L + posn] : posn;
+      }
+      continue;
+    }
     int run_sel = sel_start, run_eq = S.off_eq[t][warp];
-    // one selection: the warp's picks are compacted in order into its own part
-    // of the key buffer (never past the keys it has read), then copied out
-    // with coalesced stores; two selections: stored directly
-    const bool stage = p.ntracks == 1;
-    // every key equal to T is taken (the usual case): no ranks among equal keys
-    const bool simple = all[t] || take[t] >= S.eqtot[t];
-    const uint32_t thr = all[t] ? 1u : T[t];
     const unsigned lt = (1u << lane) - 1u;
     for (int b0 = w_lo; b0 < w_hi; b0 += 128) {
       const int i = b0 + 4 * lane;
       const uint4 k4 = *reinterpret_cast<const uint4*>(keys + i);
       const uint32_t kv[4] = {k4.x, k4.y, k4.z, k4.w};
-      int sel_m = 0;                           // bit u: key u is taken
-      int warp_eq = 0;
-      if (simple) {
+      int sel_m = 0, eq_m = 0;                 // bit u: key u is above / equal to T
 #pragma unroll
-        for (int u = 0; u < 4; ++u) sel_m |= (kv[u] >= thr && i + u < w_hi) << u;
-        if (!__any_sync(0xffffffffu, sel_m)) continue;
-      } else {
-        int eq_m = 0;                          // bit u: key u equals T
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const bool valid = kv[u] != 0u && i + u < w_hi;
-          sel_m |= (valid && kv[u] > T[t]) << u;
-          eq_m |= (valid && kv[u] == T[t]) << u;
-        }
-        // position order is lane-major: the keys of lower lanes, then this
-        // lane's earlier keys, come first
-        int eq_lower = 0;
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const unsigned eb = __ballot_sync(0xffffffffu, (eq_m >> u) & 1);
-          eq_lower += __popc(eb & lt);
-          warp_eq += __popc(eb);
-        }
-        int rank = run_eq + eq_lower;
-#pragma unroll
-        for (int u = 0; u < 4; ++u)
-          if ((eq_m >> u) & 1) {
-            if (rank < take[t]) sel_m |= 1 << u;
-            ++rank;
-          }
+      for (int u = 0; u < 4; ++u) {
+        const bool valid = kv[u] != 0u && i + u < w_hi;
+        sel_m |= (valid && (all[t] || kv[u] > T[t])) << u;
+        eq_m |= (valid && !all[t] && kv[u] == T[t]) << u;
       }
+      // position order is lane-major: the keys of lower lanes, then this
+      // lane's earlier keys, come first
+      int eq_lower = 0, warp_eq = 0;
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const unsigned eb = __ballot_sync(0xffffffffu, (eq_m >> u) & 1);
+        eq_lower += __popc(eb & lt);
+        warp_eq += __popc(eb);
+      }
+      int rank = run_eq + eq_lower;
+#pragma unroll
+      for (int u = 0; u < 4; ++u)
+        if ((eq_m >> u) & 1) {
+          if (rank < take[t]) sel_m |= 1 << u;
+          ++rank;
+        }
       int sel_lower = 0, warp_sel = 0;
 #pragma unroll
       for (int u = 0; u < 4; ++u) {
@@ -393,22 +419,11 @@ __global__ void __launch_bounds__(NT, 1) topk_cta_kernel(CtaParams p) {
 #pragma unroll
       for (int u = 0; u < 4; ++u)
         if ((sel_m >> u) & 1) {
-          if (stage)
-            keys[w_lo + (pos - sel_start)] = static_cast<uint32_t>(i + u);
-          else if (pos < p.count[t])
-            o[pos] = p.ids ? p.ids[r * p.L + i + u] : i + u;
+          if (pos < p.count[t]) o[pos] = p.ids ? p.ids[r * p.L + i + u] : i + u;
           ++pos;
         }
       run_sel += warp_sel;
       run_eq += warp_eq;
-    }
-    if (stage) {
-      __syncwarp();
-      for (int j = lane; j < run_sel - sel_start; j += 32) {
-        const int q = sel_start + j;
-        const int posn = static_cast<int>(keys[w_lo + j]);
-        if (q < p.count[t]) o[q] = p.ids ? p.ids[r * p.L + posn] : posn;
-      }
     }
   }
   // padding: positions beyond the selectable keys
