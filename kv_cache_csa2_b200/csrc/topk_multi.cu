@@ -49,6 +49,7 @@ constexpr int kTracks = 2;
 constexpr int kMaxRowsMulti = 1024;
 constexpr int kMaxC = 64;
 constexpr int kCandCap = 4096;            // candidate keys per row and selection
+static_assert(kCandCap % 512 == 0 && kCandCap < (1 << 15), "candidates per thread; packed counts");
 
 struct SelParams {
   const float* scores;
@@ -125,13 +126,13 @@ __device__ __forceinline__ bool row_barrier(unsigned* ctr, unsigned target, int*
   return !*abort_s;
 }
 
-__global__ void __launch_bounds__(kT) topk_multi_kernel(SelParams p) {
+__global__ void __launch_bounds__(kT, 2) topk_multi_kernel(SelParams p) {
   extern __shared__ uint32_t keys[];
   __shared__ int hist_s[kTracks][kBins];
   __shared__ int ws[33];
   __shared__ uint32_t sh_min, sh_max;
   __shared__ int sh_bin[kTracks], sh_above[kTracks], sh_total[kTracks];
-  __shared__ int sh_off[kTracks], sh_take[kTracks], sh_all_sel[kTracks];
+  __shared__ int sh_off[kTracks], sh_take[kTracks], sh_all_sel[kTracks], sh_eqin[kTracks];
   __shared__ int seg_gt[kTracks][kT / 32], seg_eq[kTracks][kT / 32];
   __shared__ int abort_s;
   const int tid = threadIdx.x;
@@ -331,34 +332,53 @@ __global__ void __launch_bounds__(kT) topk_multi_kernel(SelParams p) {
       uint32_t* ck = p.ckey + r * kTracks * kCandCap;
       int32_t* cp = p.cpos + r * kTracks * kCandCap;
       int* cc = p.ccnt + r * kTracks;
-      for (int t = 0; t < p.ntracks; ++t) {
-        const uint32_t bin_max = prefix[t] | ~mask[t];
-        int above = 0;
-        for (int i0 = 0; i0 < n; i0 += kT) {
+      {
+        uint32_t bin_max[kTracks];
+#pragma unroll
+        for (int t = 0; t < kTracks; ++t) bin_max[t] = prefix[t] | ~mask[t];
+        int above[kTracks] = {0, 0};
+        for (int i0 = 0; i0 < n; i0 += kT) {                 // one sweep serves both selections
           const int i = i0 + tid;
           const uint32_t key = i < n ? keys[i] : 0u;
-          const bool sel = key != 0u && (all[t] || key > bin_max);
-          const bool in_bin = key != 0u && !all[t] && (key & mask[t]) == prefix[t];
-          above += sel ? 1 : 0;
-          const unsigned bal = __ballot_sync(0xffffffffu, in_bin);
-          int base = 0;
-          if (lane == 0 && bal) base = atomicAdd(&cc[t], __popc(bal));
-          base = __shfl_sync(0xffffffffu, base, 0);
-          if (in_bin) {
-            const int idx = base + __popc(bal & ((1u << lane) - 1u));
-            ck[t * kCandCap + idx] = key;
-            cp[t * kCandCap + idx] = static_cast<int32_t>(lo + i);
+#pragma unroll
+          for (int t = 0; t < kTracks; ++t) {
+            if (t >= p.ntracks) break;
+            above[t] += (key != 0u && (all[t] || key > bin_max[t])) ? 1 : 0;
+            const bool in_bin = key != 0u && !all[t] && (key & mask[t]) == prefix[t];
+            const unsigned bal = __ballot_sync(0xffffffffu, in_bin);
+            if (bal) {                                       // rare: the threshold bin is small
+              int base = 0;
+              if (lane == 0) base = atomicAdd(&cc[t], __popc(bal));
+              base = __shfl_sync(0xffffffffu, base, 0);
+              if (in_bin) {
+                const int idx = base + __popc(bal & ((1u << lane) - 1u));
+                ck[t * kCandCap + idx] = key;
+                cp[t * kCandCap + idx] = static_cast<int32_t>(lo + i);
+              }
+            }
           }
         }
-        int tot;
-        block_scan(above, ws, &tot);
-        if (tid == 0) cr[(c * kTracks + t) * 2] = tot;
+        for (int t = 0; t < p.ntracks; ++t) {
+          int tot;
+          block_scan(above[t], ws, &tot);
+          if (tid == 0) cr[(c * kTracks + t) * 2] = tot;
+        }
       }
       ok = row_barrier(ctr, C * (++epoch), p.err, &abort_s);
       // (2) every CTA refines the threshold over the candidates (same result)
       for (int t = 0; t < p.ntracks && ok; ++t) {
         if (all[t]) continue;
         const int nc = __ldcg(&cc[t]);
+        // this thread's candidates (nc <= kCandCap = 8 per thread), loaded once
+        constexpr int kPer = kCandCap / kT;
+        uint32_t ckr[kPer];
+        int32_t cpr[kPer];
+#pragma unroll
+        for (int u = 0; u < kPer; ++u) {
+          const int i = tid + u * kT;
+          ckr[u] = i < nc ? __ldcg(&ck[t * kCandCap + i]) : 0u;
+          cpr[u] = i < nc ? __ldcg(&cp[t * kCandCap + i]) : -1;
+        }
         int lb = lowbit;
         while (lb > 0) {
           const int width = lb >= kDigit ? kDigit : lb;
@@ -366,10 +386,10 @@ __global__ void __launch_bounds__(kT) topk_multi_kernel(SelParams p) {
           const int bins = 1 << width;
           for (int i = tid; i < kBins; i += kT) hist_s[t][i] = 0;
           __syncthreads();
-          for (int i = tid; i < nc; i += kT) {
-            const uint32_t key = __ldcg(&ck[t * kCandCap + i]);
-            if ((key & mask[t]) == prefix[t]) atomicAdd(&hist_s[t][(key >> shift) & (bins - 1)], 1);
-          }
+#pragma unroll
+          for (int u = 0; u < kPer; ++u)
+            if (cpr[u] >= 0 && (ckr[u] & mask[t]) == prefix[t])
+              atomicAdd(&hist_s[t][(ckr[u] >> shift) & (bins - 1)], 1);
           __syncthreads();
           const int per = (bins + kT - 1) / kT;
           int h[kBins / kT];
@@ -402,24 +422,26 @@ __global__ void __launch_bounds__(kT) topk_multi_kernel(SelParams p) {
         // the lower chunks' counts above the bin and the candidates' positions
         const uint32_t Tt = prefix[t];
         int gt_b = 0, eq_b = 0, eq_in = 0;
-        for (int i = tid; i < nc; i += kT) {
-          const uint32_t key = __ldcg(&ck[t * kCandCap + i]);
-          const int64_t pos = __ldcg(&cp[t * kCandCap + i]);
+#pragma unroll
+        for (int u = 0; u < kPer; ++u) {
+          const int64_t pos = cpr[u];
+          if (pos < 0) continue;
           if (pos < lo) {
-            gt_b += key > Tt ? 1 : 0;
-            eq_b += key == Tt ? 1 : 0;
+            gt_b += ckr[u] > Tt ? 1 : 0;
+            eq_b += ckr[u] == Tt ? 1 : 0;
           } else if (pos < lo + n) {
-            eq_in += key == Tt ? 1 : 0;
+            eq_in += ckr[u] == Tt ? 1 : 0;
           }
         }
         for (int cc2 = tid; cc2 < c; cc2 += kT) gt_b += __ldcg(&cr[(cc2 * kTracks + t) * 2]);
-        int tg, te, ti;
+        int tg, tp;
         block_scan(gt_b, ws, &tg);
-        block_scan(eq_b, ws, &te);
-        block_scan(eq_in, ws, &ti);
+        block_scan(eq_b | (eq_in << 16), ws, &tp);          // both counts <= kCandCap < 2^16
+        const int te = tp & 0xffff, ti = tp >> 16;
         if (tid == 0) {
           sh_off[t] = tg + min(te, kk[t]);
           sh_take[t] = max(0, min(kk[t] - te, ti));
+          sh_eqin[t] = ti;
           sh_all_sel[t] = p.count[t];
         }
       }
@@ -452,6 +474,43 @@ __global__ void __launch_bounds__(kT) topk_multi_kernel(SelParams p) {
       }
     }
 
+    // Candidate path, every selection taking all of this chunk's keys equal to
+    // its T: one sweep per selection compacts the picks, in order, into the
+    // (now free) histogram space, then per-warp offsets and coalesced copies.
+    bool simple = use_cand && ok;
+    for (int t = 0; t < p.ntracks; ++t)
+      if (!all[t] && sh_take[t] != sh_eqin[t]) simple = false;
+    if (simple) {
+      const unsigned ltm = (1u << lane) - 1u;
+      const int sseg = (((n + kT / 32 - 1) / (kT / 32)) + 31) & ~31;
+      const int s_lo = std::min(n, warp * sseg), s_hi = std::min(n, s_lo + sseg);
+      int* stage = &hist_s[0][0];                 // kTracks * kBins >= n ints
+      for (int t = 0; t < p.ntracks; ++t) {
+        const uint32_t thr = all[t] ? 1u : prefix[t];
+        int cnt = 0;
+        for (int i0 = s_lo; i0 < s_hi; i0 += 32) {
+          const int i = i0 + lane;
+          const uint32_t key = i < s_hi ? keys[i] : 0u;
+          const bool sel = key >= thr;
+          const unsigned sb = __ballot_sync(0xffffffffu, sel);
+          if (sel) stage[s_lo + cnt + __popc(sb & ltm)] = static_cast<int>(lo + i);
+          cnt += __popc(sb);
+        }
+        if (lane == 0) seg_gt[t][warp] = cnt;
+        __syncthreads();
+        int before = 0;
+        for (int w2 = 0; w2 < warp; ++w2) before += seg_gt[t][w2];
+        int32_t* o = p.out[t] + r * static_cast<int64_t>(p.count[t]);
+        for (int j = lane; j < cnt; j += 32) {
+          const int q = sh_off[t] + before + j;
+          const int posn = stage[s_lo + j];
+          if (q < p.count[t]) o[q] = p.ids ? p.ids[r * p.L + posn] : posn;
+        }
+        if (c == C - 1)
+          for (int q = sh_all_sel[t] + tid; q < p.count[t]; q += kT) o[q] = -1;
+        __syncthreads();
+      }
+    } else {
     // per-chunk counts of keys above / equal to each threshold, per warp
     // segment (16 contiguous segments of the chunk, one per warp)
     const unsigned lt_mask = (1u << lane) - 1u;
@@ -535,6 +594,7 @@ __global__ void __launch_bounds__(kT) topk_multi_kernel(SelParams p) {
           for (int q = sh_all_sel[t] + tid; q < p.count[t]; q += kT) o[q] = -1;
       }
     }
+    }  // not simple
     __syncthreads();
   }
 }
