@@ -167,6 +167,22 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int64_t n_waves = (p.n_queries - slot + p.G - 1) / p.G;
   constexpr uint32_t S_COL = 0;                       // S at columns [0, 64)
   constexpr uint32_t O_COL = 256;                     // O^T chunk mc at [256 + 64 mc, ...)
+  // gather mapping (warps 2-5): thread et copies 16-byte chunk c16 of rows
+  // grow0 + 16 i (i < 8) in every 64-column block; eight consecutive threads
+  // cover one 128-byte row segment
+  const int et = (warp - 2) * 32 + lane;
+  const int c16 = et & 7, grow0 = et >> 3;
+  // the first wave's row ids, loaded while the barriers and TMEM are set up
+  pdl_wait();                                  // the selection comes from the kernel before
+  int32_t first_ids[8];
+  if (warp >= 2 && n_waves > 0) {
+    const int32_t* ids = p.topk + static_cast<int64_t>(slot) * p.k;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int64_t pos = static_cast<int64_t>(tile) * kRows + grow0 + 16 * i;
+      first_ids[i] = pos < p.k ? ids[pos] : -1;
+    }
+  }
 
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
@@ -188,7 +204,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  pdl_wait();                                  // the selection comes from the kernel before
 
   if (warp == 0) {
     // ------------------------------------------------------------ q loader
@@ -251,22 +266,18 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int quad = warp & 3;
     const int ew = warp - 2;                           // epilogue warp 0..3
     const int row = quad * 32 + lane;                  // TMEM lane = tile row
-    const int et = ew * 32 + lane;                     // epilogue thread 0..127
     const uint32_t lane_off = static_cast<uint32_t>(quad * 32) << 16;
     const int hb = reduced_head_base(lane);
-    // gather: thread et copies 16-byte chunk c16 of rows grow0 + 16 i (i < 8)
-    // in every 64-column block; eight consecutive threads cover one 128-byte
-    // row segment.  (grow0 + 16 i) & 7 == grow0 & 7: one swizzle per thread.
-    const int c16 = et & 7, grow0 = et >> 3;
+    // (grow0 + 16 i) & 7 == grow0 & 7: one swizzle per thread
     const uint32_t swz = static_cast<uint32_t>((c16 ^ (grow0 & 7)) << 4);
-    auto issue_gather = [&](int64_t qi) {
+    auto issue_gather = [&](int64_t qi, const int32_t* pre) {   // pre: this wave's ids, or null
       const uint16_t* base = p.kv + (qi / p.Q) * p.n * DV + c16 * 8;
       const int32_t* ids = p.topk + qi * p.k;
       int64_t off[8];
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
         const int64_t pos = static_cast<int64_t>(tile) * kRows + grow0 + 16 * i;
-        int id = pos < p.k ? ids[pos] : -1;
+        int id = pre ? pre[i] : (pos < p.k ? ids[pos] : -1);
         if (id >= p.n || id < -1) {
           raise_dev_error(p.err, DEVERR_BOUNDS);
           id = -1;
@@ -292,7 +303,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #undef CSA2_PUBLISH
     };
     if (n_waves > 0) {
-      issue_gather(slot);
+      issue_gather(slot, first_ids);
       publish_gather();
     }
     bool ok = true;
@@ -549,7 +560,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
         epi_bar();
-        if (more && ds + kStageDims >= d1) issue_gather(qi + p.G);   // the KV region is free again
+        if (more && ds + kStageDims >= d1) issue_gather(qi + p.G, nullptr);   // the KV region is free again
         // normalise, bf16, 8-byte stores of 4 dims
         const int pieces = nd / 4;
         for (int i = et; i < HA * pieces; i += 128) {
@@ -564,7 +575,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         epi_bar();
       }
-      if (more && d1 <= d0) issue_gather(qi + p.G);
+      if (more && d1 <= d0) issue_gather(qi + p.G, nullptr);
       if (tile == 0 && p.lse && et < HA)
         p.lse[qi * HA + et] = sML2[HA + et] > 0.0f ? sML2[et] + logf(sML2[HA + et]) : -INFINITY;
       // this CTA alone reads its dims of every partial: drop those lines from L2
