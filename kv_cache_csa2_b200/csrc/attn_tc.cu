@@ -8,12 +8,13 @@
 // cut into T = ceil(k / 128) tiles of 128 rows and each (query, tile) unit runs
 // on one CTA.  The CTA computes its tile's partial result with the tile's own
 // per-head max m (P = exp(s - m) rounded to bf16, l = sum of P, O = P^T KV in
-// f32), writes (O, m, l) to a global workspace and meets the query's other
-// T - 1 CTAs at a counter in global memory.  CTA t then reduces output dims
-// [t * dpc, (t + 1) * dpc) over the T partials in tile order, each weighted by
+// f32), writes (O, m, l) to a global workspace and raises its flag (a count
+// of the partials it has written).  CTA t then reduces output dims
+// [t * dpc, (t + 1) * dpc) over the T partials in tile order -- partial j is
+// fetched as soon as tile j's flag shows it --, each weighted by
 // exp(m_j - M) with M = max_j m_j, divides by L = sum_j l_j exp(m_j - M) and
 // writes bf16 out (tile 0 also lse = M + log L).  The launch is cooperative:
-// the whole grid is resident, so the counter wait always ends.  A grid holds
+// the whole grid is resident, so every flag wait ends.  A grid holds
 // the units of G queries and loops over the batch in waves of G queries.  The
 // split and the reduction order depend on k only, so results are
 // deterministic and batch-invariant.
@@ -27,8 +28,8 @@
 //   warps 2-5  gather of the tile's 128 rows (16-byte cp.async copies straight
 //              into the 128-byte-swizzled layout, 64 per thread in flight; the
 //              next wave's gather is issued as soon as this wave's products are
-//              done), softmax, partial write, counter wait, reduction, output.
-// Every wait is bounded (mbarriers 2 s, the counter 1 s); a CTA that gives up
+//              done), softmax, partial write, flag waits, reduction, output.
+// Every wait is bounded (mbarriers 2 s, the flags 1 s); a CTA that gives up
 // records CSA2_ERR_TIMEOUT and still takes every later step, so no other CTA
 // waits for it in vain.
 #include <algorithm>
@@ -79,7 +80,7 @@ struct Params {
   uint16_t* out;                   // [B*Q, 64, 512]
   float* lse;                      // [B*Q, 64] or null
   float* part;                     // [2][grid][kSlotFloats]
-  unsigned long long* sync;        // [G] arrival counters (multiples of T between launches)
+  unsigned* flag;                  // [grid] partials written per CTA (equal across a query's CTAs between waves)
   int* err;
   int64_t n, n_queries;
   int Q, k, T, G, dpc;
@@ -125,9 +126,9 @@ __device__ __forceinline__ float rescale(float m, float M) {
   return (m == -INFINITY || M == -INFINITY) ? 0.0f : __expf(m - M);
 }
 
-__device__ __forceinline__ unsigned long long ld_acquire_u64(const unsigned long long* p) {
-  unsigned long long v;
-  asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+__device__ __forceinline__ unsigned ld_acquire_u32(const unsigned* p) {
+  unsigned v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
   return v;
 }
 
@@ -140,6 +141,7 @@ __device__ __forceinline__ void discard_l2_line(const void* p) {
 __global__ void __launch_bounds__(kThreads, 1)
     attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const Params p) {
   extern __shared__ uint8_t smem_raw[];
+  __shared__ unsigned sh_gen;
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sKV = smem + OFF_KV;
   uint8_t* sP = smem + OFF_P;
@@ -407,38 +409,38 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       tc_fence_before();
-      if (et == 0) {
-        bulk_wait_all();
-        fence_proxy_async_global();
-        __threadfence();
-      }
       const int64_t base = buf + (blockIdx.x - tile);  // workspace slot of tile 0
       const float* pb = p.part + base * kSlotFloats;   // slot j at pb + j * kSlotFloats
       const int d0 = min(DV, tile * p.dpc), d1 = min(DV, d0 + p.dpc);
       const uint32_t slice_bytes = static_cast<uint32_t>(d1 - d0) * HA * 4;
       if (et == 0) {
-        // meet the query's other CTAs (all resident: the launch is cooperative)
-        unsigned long long* cnt = p.sync + slot;
-        const unsigned long long old = atomicAdd(cnt, 1ull);
-        const unsigned long long target = (old / p.T + 1) * p.T;
+        bulk_wait_all();
+        fence_proxy_async_global();
+        __threadfence();
+        // publish: this CTA's flag counts the partials it has written
+        sh_gen = atomicAdd(&p.flag[blockIdx.x], 1u) + 1u;
+        if (p.bulk) mbar_arrive_expect_tx(r_full, (slice_bytes + 2 * HA * 4) * p.T);
+      }
+      epi_bar();
+      // thread j waits for tile j's partial of this wave (every CTA of the grid
+      // is resident: the launch is cooperative) and, on the bulk path, loads
+      // this CTA's dims of it and its (m, l) at once
+      if (et < p.T) {
+        const unsigned gen = sh_gen;
+        const unsigned* fj = p.flag + (blockIdx.x - tile) + et;
         const uint64_t t0 = globaltimer_ns();
-        while (ld_acquire_u64(cnt) < target) {
+        while (static_cast<int>(ld_acquire_u32(fj) - gen) < 0) {
           if (globaltimer_ns() - t0 > 1000000000ull) {
             raise_dev_error(p.err, DEVERR_TIMEOUT);
             *abort_flag = 1;
             break;
           }
         }
-        __threadfence();
         fence_proxy_async_global();
         if (p.bulk) {
-          // this CTA's dims of every partial into the KV region, every (m, l) into the P region
-          mbar_arrive_expect_tx(r_full, (slice_bytes + 2 * HA * 4) * p.T);
-          for (int j = 0; j < p.T; ++j) {
-            const float* sj = pb + static_cast<int64_t>(j) * kSlotFloats;
-            if (slice_bytes > 0) bulk_load(sKV + j * slice_bytes, sj + d0 * HA, slice_bytes, r_full);
-            bulk_load(sP + j * 2 * HA * 4, sj + kPartFloats, 2 * HA * 4, r_full);
-          }
+          const float* sj = pb + static_cast<int64_t>(et) * kSlotFloats;
+          if (slice_bytes > 0) bulk_load(sKV + et * slice_bytes, sj + d0 * HA, slice_bytes, r_full);
+          bulk_load(sP + et * 2 * HA * 4, sj + kPartFloats, 2 * HA * 4, r_full);
         }
       }
       epi_bar();
@@ -646,7 +648,7 @@ WsLayout ws_layout(int64_t n_queries, Shape s) {
   const int64_t ctas = g * s.T;
   WsLayout l;
   l.part = a256(static_cast<size_t>(2 * ctas) * kSlotFloats * 4);
-  l.sync = a256(static_cast<size_t>(g) * 8);
+  l.sync = a256(static_cast<size_t>(ctas) * 4);
   l.total = l.part + l.sync;
   return l;
 }
@@ -687,8 +689,8 @@ csa2_status launch_sparse_attn_tc(const void* q, const csa2_kv& kv, const int32_
   p.out = static_cast<uint16_t*>(out);
   p.lse = lse;
   p.part = static_cast<float*>(ws);
-  p.sync = sync_zeroed ? sync_zeroed
-                       : reinterpret_cast<unsigned long long*>(static_cast<char*>(ws) + lay.part);
+  p.flag = sync_zeroed ? reinterpret_cast<unsigned*>(sync_zeroed)
+                       : reinterpret_cast<unsigned*>(static_cast<char*>(ws) + lay.part);
   p.err = device_error_word();
   p.n = kv.n;
   p.n_queries = n_queries;
@@ -699,10 +701,10 @@ csa2_status launch_sparse_attn_tc(const void* q, const csa2_kv& kv, const int32_
   p.dpc = s.dpc;
   p.bulk = static_cast<int64_t>(s.T) * s.dpc * HA * 4 <= kKB * kKBBytes && s.T * 2 * HA * 4 <= kRows * 128;
   p.scale = scale;
-  if (!sync_zeroed) {          // a caller workspace: counters start at zero
+  if (!sync_zeroed) {          // a caller workspace: flags start at zero
     begin_launch(stream);
-    if (cudaMemsetAsync(p.sync, 0, static_cast<size_t>(G) * 8, stream) != cudaSuccess)
-      return check_launch("sparse_attn_tc: clear counters");
+    if (cudaMemsetAsync(p.flag, 0, static_cast<size_t>(G) * s.T * 4, stream) != cudaSuccess)
+      return check_launch("sparse_attn_tc: clear flags");
     note_launch(LK_OTHER, 1, stream);
   }
   cudaLaunchConfig_t cfg = {};

@@ -42,9 +42,9 @@ csa2_status launch_select_topk(const float* scores, int64_t rows, int64_t L, int
 constexpr int kAttnMaxGrid = 160;
 
 size_t sparse_attn_workspace(int B, int Q, int Ha, int D, int k, csa2_kv_fmt fmt);
-// sync_zeroed: kAttnMaxGrid arrival counters that were zero before their
-// first use and are left consistent by every launch (a layer group's), or
-// NULL to take them from the workspace and clear them on the stream.
+// sync_zeroed: kAttnMaxGrid * 8 bytes of per-CTA flags that were zero before
+// their first use and are left consistent by every launch (a layer group's),
+// or NULL to take them from the workspace and clear them on the stream.
 csa2_status launch_sparse_attn(const void* q, const csa2_kv& kv, const int32_t* topk, int B,
                                int Q, int Ha, int k, float scale, void* out, float* lse, void* ws,
                                size_t ws_bytes, unsigned long long* sync_zeroed,
