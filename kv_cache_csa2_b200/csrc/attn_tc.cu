@@ -62,7 +62,7 @@ constexpr int OFF_RED = OFF_Q + kKB * HA * 128;        // [4 warps][HA] f32
 constexpr int OFF_ML = OFF_RED + 4 * HA * 4;           // this tile's m[HA], l[HA]
 constexpr int OFF_ML2 = OFF_ML + 2 * HA * 4;           // the query's M[HA], L[HA]
 constexpr int OFF_BAR = OFF_ML2 + 2 * HA * 4;
-constexpr int NBAR = 16;
+constexpr int NBAR = 20;
 constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
 constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;
 // reduction scratch inside the q region: output staging [HA][kStageStride]
@@ -156,7 +156,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* q_full = bar + 0;
   uint64_t* s_full = bar + 1;
   uint64_t* p_full = bar + 2;
-  uint64_t* o_full = bar + 3;
+  uint64_t* o_full = bar + 16;                 // [4]: one per 128-dim chunk of O^T
   uint64_t* m_done = bar + 4;                  // the reduction no longer needs the q region
   uint64_t* r_full = bar + 5;                  // this CTA's dims of every partial are in the KV region
   uint64_t* kv_full = bar + 8;                 // [8]: one per 64-column block of the tile
@@ -190,7 +190,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(q_full, 1);
     mbar_init(s_full, 1);
     mbar_init(p_full, 4);
-    mbar_init(o_full, 1);
+    for (int mc = 0; mc < 4; ++mc) mbar_init(&o_full[mc], 1);
     mbar_init(m_done, 1);
     mbar_init(r_full, 1);
     for (int kb = 0; kb < kKB; ++kb) mbar_init(&kv_full[kb], 128);
@@ -253,13 +253,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!mbar_wait(p_full, par, abort_flag, p.err)) break;
         tc_fence_after();
 #pragma unroll
-        for (int mc = 0; mc < 4; ++mc)
+        for (int mc = 0; mc < 4; ++mc) {
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk)
             mma_bf16(tmem + O_COL + 64 * mc,
                      desc_mnmajor_sw128(kv0 + 2 * mc * kKBBytes + kk * 2048, kKBBytes, 1024),
                      desc_mnmajor_sw128(p0 + kk * 2048, 8192, 1024), idesc_o, kk != 0);
-        mma_commit(o_full);
+          mma_commit(&o_full[mc]);                 // chunk mc can be read while mc+1 computes
+        }
       }
     }
     __syncwarp();
@@ -379,8 +380,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       // O^T is staged in the KV region as [dim][16 chunks of 4 heads] with
       // chunk h4 at position h4 ^ (dim & 7) (conflict-free) and written with
       // (m, l) by two bulk stores; the slot keeps that layout.
-      ok = ok && mbar_wait(o_full, par, abort_flag, p.err);
-      tc_fence_after();
       const bool more = w + 1 < n_waves;
       const int64_t buf = (w & 1) * static_cast<int64_t>(gridDim.x);
       const uint32_t kv0 = smem_u32(sKV);
@@ -389,6 +388,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int mc = 0; mc < 4; ++mc) {
         const int dim = mc * 128 + row;
         const uint32_t srow = kv0 + dim * (HA * 4);
+        // chunk mc's products are done; its staging rows are the KV blocks
+        // 2mc, 2mc+1, which only chunk mc's products read
+        ok = ok && mbar_wait(&o_full[mc], par, abort_flag, p.err);
+        tc_fence_after();
         if (ok) {
           uint32_t v0[32], v1[32];
           tmem_ld32(tmem + lane_off + O_COL + 64 * mc, v0);
