@@ -395,11 +395,14 @@ csa2_status csa2_index_topk(csa2_mode mode, const void* q, const float* w, const
   const size_t sbytes = align256(static_cast<size_t>(rows) * L * sizeof(float));
   void* sel_ws = static_cast<char*>(workspace) + sbytes;
   const size_t sel_bytes = workspace_bytes - sbytes;
-  // the dual selection's counters are cleared first, so that it follows the
-  // scoring kernel directly (programmatic dependent launch)
-  if (pool_out) CSA2_TRY(select_topk_clear(rows, L, sel_ws, sel_bytes, s));
+  // the dual selection's counters are cleared by the scoring kernel (or else
+  // just after it), so that the selection follows that kernel directly
+  // (programmatic dependent launch)
+  ClearOnLaunch clear;
+  if (pool_out) clear = select_topk_clear_region(rows, L, sel_ws, sel_bytes);
   CSA2_TRY(launch_index_scores(q, w, k, B, Q, H, d, N, n_visible, pool_in, pool_in ? P_in : 0, act,
-                               scores, s));
+                               scores, s, clear.ptr ? &clear : nullptr));
+  if (pool_out && clear.ptr && !clear.done) CSA2_TRY(select_topk_clear(rows, L, sel_ws, sel_bytes, s));
   if (pool_out) {
     // the pool and the top-k in the same selection passes when the kernel applies
     const csa2_status st = launch_select_topk2(scores, rows, L, k_top, nullptr, topk_out, P_out,

@@ -17,7 +17,7 @@ namespace csa2 {
 csa2_status launch_index_scores_tc(const void* q, const float* w, const void* k, int B, int Q,
                                    int H, int d, int64_t N, const int32_t* n_visible,
                                    const int32_t* pool, int P, csa2_index_act act, float* scores,
-                                   cudaStream_t stream);
+                                   cudaStream_t stream, ClearOnLaunch* clear);
 
 namespace {
 
@@ -126,11 +126,12 @@ csa2_status launch_index_scores_simt(const void* q, const float* w, const void* 
 
 csa2_status launch_index_scores(const void* q, const float* w, const void* k, int B, int Q, int H,
                                 int d, int64_t N, const int32_t* n_visible, const int32_t* pool,
-                                int P, csa2_index_act act, float* scores, cudaStream_t stream) {
+                                int P, csa2_index_act act, float* scores, cudaStream_t stream,
+                                ClearOnLaunch* clear) {
   const int64_t L = pool ? P : N;
   if (L == 0 || B == 0 || Q == 0) return CSA2_OK;
   csa2_status s = launch_index_scores_tc(q, w, k, B, Q, H, d, N, n_visible, pool, P, act, scores,
-                                         stream);
+                                         stream, clear);
   if (s != CSA2_ERR_UNSUPPORTED) return s;
   return launch_index_scores_simt(q, w, k, B, Q, H, d, N, n_visible, pool, P, act, scores, stream);
 }

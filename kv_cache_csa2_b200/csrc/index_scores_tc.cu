@@ -53,6 +53,8 @@ struct Params {
   int64_t N;
   int relu;
   int q_tma;          // queries by TMA (one query per group, no padded heads)
+  uint32_t* clear;    // words CTA 0 zeroes at start for the next kernel, or null
+  int clear_words;
   int n_qgroups, n_tiles;
   int64_t n_units;
 };
@@ -106,6 +108,8 @@ __global__ void __launch_bounds__(POOL ? kPoolThreads : kThreads, 1)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t L = POOL ? p.P : p.N;
   pdl_release();                               // the selection kernel may start launching
+  if (blockIdx.x == 0 && p.clear)              // the selection's counters (read after this kernel)
+    for (int i = threadIdx.x; i < p.clear_words; i += blockDim.x) p.clear[i] = 0u;
 
   // balanced contiguous range of units for this CTA
   const int64_t u0 = p.n_units * blockIdx.x / gridDim.x;
@@ -381,7 +385,7 @@ __global__ void __launch_bounds__(POOL ? kPoolThreads : kThreads, 1)
 template <int DK, int NQ, int HP, bool POOL>
 csa2_status run_tc(const void* q, const float* w, const void* k, int B, int Q, int H, int64_t N,
                    const int32_t* n_visible, const int32_t* pool, int P, csa2_index_act act,
-                   float* scores, cudaStream_t stream) {
+                   float* scores, cudaStream_t stream, ClearOnLaunch* clear) {
   using C = Cfg<DK, NQ, HP, POOL>;
   CUtensorMap map;
   memset(&map, 0, sizeof(map));
@@ -407,6 +411,8 @@ csa2_status run_tc(const void* q, const float* w, const void* k, int B, int Q, i
   p.N = N;
   p.relu = act == CSA2_ACT_RELU ? 1 : 0;
   p.q_tma = q_tma ? 1 : 0;
+  p.clear = clear ? clear->ptr : nullptr;
+  p.clear_words = clear ? clear->words : 0;
   p.n_qgroups = (Q + NQ - 1) / NQ;
   const int64_t L = POOL ? P : N;
   p.n_tiles = static_cast<int>((L + kTileRows - 1) / kTileRows);
@@ -422,7 +428,9 @@ csa2_status run_tc(const void* q, const float* w, const void* k, int B, int Q, i
   begin_launch(stream);
   kern<<<static_cast<unsigned>(grid), POOL ? kPoolThreads : kThreads, C::BYTES, stream>>>(map, qmap, p);
   note_launch(POOL ? LK_INDEX_POOL : LK_INDEX, 1, stream);
-  return check_launch("index_scores_tc");
+  const csa2_status st = check_launch("index_scores_tc");
+  if (st == CSA2_OK && clear) clear->done = true;
+  return st;
 }
 
 }  // namespace
@@ -430,31 +438,31 @@ csa2_status run_tc(const void* q, const float* w, const void* k, int B, int Q, i
 csa2_status launch_index_scores_tc(const void* q, const float* w, const void* k, int B, int Q,
                                    int H, int d, int64_t N, const int32_t* n_visible,
                                    const int32_t* pool, int P, csa2_index_act act, float* scores,
-                                   cudaStream_t stream) {
+                                   cudaStream_t stream, ClearOnLaunch* clear) {
   if (getenv("CSA2_INDEX_SIMT")) return CSA2_ERR_UNSUPPORTED;   // force the CUDA-core kernel
   if ((d != 64 && d != 128) || H > 64) return CSA2_ERR_UNSUPPORTED;
   if (static_cast<int64_t>(B) * N > 0x7fffffffLL) return CSA2_ERR_UNSUPPORTED;
   const bool small = H <= 16;
   if (pool) {
     if (d == 64)
-      return small ? run_tc<64, 1, 16, true>(q, w, k, B, Q, H, N, n_visible, pool, P, act, scores, stream)
-                   : run_tc<64, 1, 64, true>(q, w, k, B, Q, H, N, n_visible, pool, P, act, scores, stream);
-    return small ? run_tc<128, 1, 16, true>(q, w, k, B, Q, H, N, n_visible, pool, P, act, scores, stream)
-                 : run_tc<128, 1, 64, true>(q, w, k, B, Q, H, N, n_visible, pool, P, act, scores, stream);
+      return small ? run_tc<64, 1, 16, true>(q, w, k, B, Q, H, N, n_visible, pool, P, act, scores, stream, clear)
+                   : run_tc<64, 1, 64, true>(q, w, k, B, Q, H, N, n_visible, pool, P, act, scores, stream, clear);
+    return small ? run_tc<128, 1, 16, true>(q, w, k, B, Q, H, N, n_visible, pool, P, act, scores, stream, clear)
+                 : run_tc<128, 1, 64, true>(q, w, k, B, Q, H, N, n_visible, pool, P, act, scores, stream, clear);
   }
   const bool many = Q >= 4;
   if (d == 64) {
     if (small)
-      return many ? run_tc<64, 16, 16, false>(q, w, k, B, Q, H, N, n_visible, nullptr, 0, act, scores, stream)
-                  : run_tc<64, 1, 16, false>(q, w, k, B, Q, H, N, n_visible, nullptr, 0, act, scores, stream);
-    return many ? run_tc<64, 4, 64, false>(q, w, k, B, Q, H, N, n_visible, nullptr, 0, act, scores, stream)
-                : run_tc<64, 1, 64, false>(q, w, k, B, Q, H, N, n_visible, nullptr, 0, act, scores, stream);
+      return many ? run_tc<64, 16, 16, false>(q, w, k, B, Q, H, N, n_visible, nullptr, 0, act, scores, stream, clear)
+                  : run_tc<64, 1, 16, false>(q, w, k, B, Q, H, N, n_visible, nullptr, 0, act, scores, stream, clear);
+    return many ? run_tc<64, 4, 64, false>(q, w, k, B, Q, H, N, n_visible, nullptr, 0, act, scores, stream, clear)
+                : run_tc<64, 1, 64, false>(q, w, k, B, Q, H, N, n_visible, nullptr, 0, act, scores, stream, clear);
   }
   if (small)
-    return many ? run_tc<128, 16, 16, false>(q, w, k, B, Q, H, N, n_visible, nullptr, 0, act, scores, stream)
-                : run_tc<128, 1, 16, false>(q, w, k, B, Q, H, N, n_visible, nullptr, 0, act, scores, stream);
-  return many ? run_tc<128, 4, 64, false>(q, w, k, B, Q, H, N, n_visible, nullptr, 0, act, scores, stream)
-              : run_tc<128, 1, 64, false>(q, w, k, B, Q, H, N, n_visible, nullptr, 0, act, scores, stream);
+    return many ? run_tc<128, 16, 16, false>(q, w, k, B, Q, H, N, n_visible, nullptr, 0, act, scores, stream, clear)
+                : run_tc<128, 1, 16, false>(q, w, k, B, Q, H, N, n_visible, nullptr, 0, act, scores, stream, clear);
+  return many ? run_tc<128, 4, 64, false>(q, w, k, B, Q, H, N, n_visible, nullptr, 0, act, scores, stream, clear)
+              : run_tc<128, 1, 64, false>(q, w, k, B, Q, H, N, n_visible, nullptr, 0, act, scores, stream, clear);
 }
 
 }  // namespace csa2

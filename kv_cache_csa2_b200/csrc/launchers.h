@@ -11,9 +11,18 @@ csa2_status launch_compress(const void* c, const float* z, const float* bias, in
                             int D, int m, int halo, void* out, int64_t out_bstride,
                             cudaStream_t stream);
 
+// Words of device memory that the scoring kernel clears at its start for the
+// selection launched after it, so that no separate memset sits between the
+// two; `done` tells whether the kernel that ran took it on.
+struct ClearOnLaunch {
+  uint32_t* ptr = nullptr;
+  int words = 0;
+  bool done = false;
+};
 csa2_status launch_index_scores(const void* q, const float* w, const void* k, int B, int Q, int H,
                                 int d, int64_t N, const int32_t* n_visible, const int32_t* pool,
-                                int P, csa2_index_act act, float* scores, cudaStream_t stream);
+                                int P, csa2_index_act act, float* scores, cudaStream_t stream,
+                                ClearOnLaunch* clear = nullptr);
 
 size_t select_topk_workspace(int64_t rows, int64_t L, int count);
 // Two selections of the same rows in one pass set (multi-CTA kernel); returns
@@ -27,6 +36,8 @@ csa2_status launch_select_topk2(const float* scores, int64_t rows, int64_t L, in
                                 bool ws_cleared = false);
 csa2_status select_topk_clear(int64_t rows, int64_t L, void* ws, size_t ws_bytes,
                               cudaStream_t stream);
+// The words select_topk_clear() would clear (ptr = NULL when there are none).
+ClearOnLaunch select_topk_clear_region(int64_t rows, int64_t L, void* ws, size_t ws_bytes);
 // One CTA per row, no workspace: rows of up to kSelectCtaMaxL scores.
 constexpr int64_t kSelectCtaMaxL = 32768;
 bool select_topk_cta_applies(int64_t rows, int64_t L);

@@ -723,6 +723,16 @@ csa2_status launch_select_topk2(const float* scores, int64_t rows, int64_t L, in
   return check_launch("select_topk_multi");
 }
 
+ClearOnLaunch select_topk_clear_region(int64_t rows, int64_t L, void* ws, size_t ws_bytes) {
+  ClearOnLaunch c;
+  if (cta_kernel_takes(rows, L) || !multi_applies(rows, L) || !ws || ws_bytes < ws_bytes_for(rows, L))
+    return c;
+  if ((L + chunk_for(L) - 1) / chunk_for(L) <= 1) return c;
+  c.ptr = static_cast<uint32_t*>(ws);
+  c.words = static_cast<int>(ws_cleared_bytes(rows) / 4);
+  return c;
+}
+
 csa2_status select_topk_clear(int64_t rows, int64_t L, void* ws, size_t ws_bytes,
                               cudaStream_t stream) {
   if (cta_kernel_takes(rows, L) || !multi_applies(rows, L) || !ws || ws_bytes < ws_bytes_for(rows, L))
