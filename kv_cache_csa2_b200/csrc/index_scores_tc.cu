@@ -8,7 +8,7 @@
 // (persistent, one per SM):
 //   warp 0     producer: per tile, the 128 key rows into a shared-memory ring
 //              (dense: one TMA tiled load per 64-column K-block; pool: a
-//              cp.async gather of the rows the pool names by warps 0, 6, 7, 8,
+//              cp.async gather of the rows the pool names by warps 0 and 6..12,
 //              zero-filled for empty slots); per query group, the queries
 //              (TMA when a group is one query of unpadded heads, else swizzled
 //              by the lanes) and head weights into one of two slots;
@@ -35,8 +35,10 @@ using namespace sm100;
 
 constexpr int kWarps = 6;
 constexpr int kThreads = kWarps * 32;
-// pool scoring gathers rows with cp.async from four producer warps (0, 6, 7, 8)
-constexpr int kPoolThreads = 9 * 32;
+// pool scoring gathers rows with cp.async from eight producer warps (0, 6..12)
+constexpr int kPoolProducers = 8 * 32;
+constexpr int kPoolThreads = 13 * 32;
+constexpr int kPoolRows = 128 * 8 / kPoolProducers;   // rows per producer thread and tile
 constexpr int kTileRows = 128;
 constexpr int kKBlockBytes = kTileRows * 128;  // 128 rows x 64 bf16
 constexpr int kLag = 3;                        // pool gathers: stages of copies kept in flight
@@ -117,7 +119,7 @@ __global__ void __launch_bounds__(POOL ? kPoolThreads : kThreads, 1)
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < S; ++i) {
-      mbar_init(&full[i], POOL ? kTileRows : 1);
+      mbar_init(&full[i], POOL ? kPoolProducers : 1);
       mbar_init(&empty[i], 1);
     }
     for (int i = 0; i < 2; ++i) {
@@ -142,25 +144,26 @@ __global__ void __launch_bounds__(POOL ? kPoolThreads : kThreads, 1)
 
   if (warp == 0 || (POOL && warp >= 6)) {
     // ---------------------------------------------------------------- producer
-    const int ptid = warp == 0 ? lane : 32 + (warp - 6) * 32 + lane;   // pool: row of the tile
+    const int ptid = warp == 0 ? lane : 32 + (warp - 6) * 32 + lane;   // pool: producer thread index
     int64_t prev_bg = -1;
     int qi = -1;
     int64_t it = 0;
     bool ok = true;
-    // pool gather: thread ptid copies 16-byte chunk c16 of rows rg + 16 i
-    // (i < 8) in every K-block, so eight consecutive lanes read one 128-byte
-    // segment; the ids of the next unit are loaded during the current one
+    // pool gather: thread ptid copies 16-byte chunk c16 of rows rg + RS i
+    // (i < kPoolRows) in every K-block, so eight consecutive lanes read one
+    // 128-byte segment; the ids of the next unit are loaded during the current one
+    constexpr int RS = kPoolProducers / 8;          // row stride between a thread's rows
     const int c16 = ptid & 7, rg = ptid >> 3;
-    auto pool_ids = [&](int64_t v, int32_t (&ids)[8]) {
+    auto pool_ids = [&](int64_t v, int32_t (&ids)[kPoolRows]) {
       const int64_t bgv = v / p.n_tiles;
       const int64_t qrow = (bgv / p.n_qgroups) * p.Q + bgv % p.n_qgroups;
 #pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        const int64_t slot_i = (v % p.n_tiles) * kTileRows + rg + 16 * i;
+      for (int i = 0; i < kPoolRows; ++i) {
+        const int64_t slot_i = (v % p.n_tiles) * kTileRows + rg + RS * i;
         ids[i] = slot_i < L ? p.pool[qrow * p.P + slot_i] : -1;
       }
     };
-    int32_t next_ids[8];
+    int32_t next_ids[kPoolRows];
     if (POOL && u0 < u1) pool_ids(u0, next_ids);
     for (int64_t u = u0; u < u1 && ok; ++u, ++it) {
       const int64_t bg = u / p.n_tiles;
@@ -235,17 +238,17 @@ __global__ void __launch_bounds__(POOL ? kPoolThreads : kThreads, 1)
         }
       } else {
         {
-          int32_t ids[8];
+          int32_t ids[kPoolRows];
 #pragma unroll
-          for (int i = 0; i < 8; ++i) ids[i] = next_ids[i];
+          for (int i = 0; i < kPoolRows; ++i) ids[i] = next_ids[i];
           if (u + 1 < u1) pool_ids(u + 1, next_ids);             // in flight during this unit
 #pragma unroll
-          for (int i = 0; i < 8; ++i) {
+          for (int i = 0; i < kPoolRows; ++i) {
             const bool valid = ids[i] >= 0 && ids[i] < p.N;
             const uint16_t* src = p.k + (static_cast<int64_t>(b) * p.N + (valid ? ids[i] : 0)) * DK + c16 * 8;
 #pragma unroll
             for (int kb = 0; kb < C::KB; ++kb)
-              cp_async_16(dst + kb * kKBlockBytes + sw128_offset(rg + 16 * i, c16), src + kb * 64, valid ? 16u : 0u);
+              cp_async_16(dst + kb * kKBlockBytes + sw128_offset(rg + RS * i, c16), src + kb * 64, valid ? 16u : 0u);
           }
         }
         cp_async_commit();
