@@ -44,6 +44,11 @@ bool select_topk_cta_applies(int64_t rows, int64_t L);
 csa2_status launch_select_topk_cta(const float* scores, int64_t rows, int64_t L, int count0,
                                    const int32_t* ids, int32_t* out0, int count1, int32_t* out1,
                                    cudaStream_t stream);
+// A cluster of 8 CTAs per row, no workspace: one selection (count1 <= 0) of
+// rows of up to 32768 scores when there are fewer rows than SMs.
+bool select_topk_cluster_applies(int64_t rows, int64_t L, int count0, int count1);
+csa2_status launch_select_topk_cluster(const float* scores, int64_t rows, int64_t L, int count,
+                                       const int32_t* ids, int32_t* out, cudaStream_t stream);
 csa2_status launch_select_topk(const float* scores, int64_t rows, int64_t L, int count,
                                const int32_t* ids, int32_t* out, void* ws, size_t ws_bytes,
                                cudaStream_t stream);

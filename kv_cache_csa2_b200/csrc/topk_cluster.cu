@@ -1,0 +1,559 @@
+// Top-k selection of short rows (up to 32768 scores) with a cluster of 8 CTAs
+// per row, for batches too small to fill the GPU with one CTA per row (the
+// hierarchical indexer's pool in a Reindex layer: 8 rows of 16384).  Sources:
+// "读完这篇，你就搞懂 DeepSeek v4 了", 闪电索引机制 (keep the k best
+// entries); "Recall之王", Hierarchical Sparse Indexer (the Reindex layer's
+// top-k inside the pool).
+//
+// Same result as the one-CTA kernel: score descending, ties to the lower
+// position, -inf and NaN never chosen, -0 ranks as +0; selected positions
+// are written in position order, padded with -1.  CTA c of a row's cluster
+// holds positions [c * chunk, (c + 1) * chunk) as order-preserving keys in
+// its shared memory.  Data moves between the CTAs by stores into the other
+// CTAs' shared memory followed by one cluster barrier (a remote load costs a
+// round trip; a store does not wait):
+//   1. each CTA's smallest / largest selectable key and count go to every CTA;
+//   2. radix passes of 8-bit digits below the bits all selectable keys share:
+//      each CTA histograms its keys and stores the histogram into every CTA,
+//      so every CTA sums the same eight histograms and takes the same bin;
+//   3. once the threshold bin holds at most kMaxCand keys, each CTA lists its
+//      keys in that bin and every CTA copies the eight lists (in CTA order);
+//      the remaining 8-bit passes run over the candidates alone;
+//   4. each CTA's output offset follows from the counts it has: the keys above
+//      the threshold bins in the CTAs before it (sent with the lists) and the
+//      candidates before its own in the copied list.  Only a row whose
+//      threshold bin never fits the list needs one more exchange of counts.
+// Integer counts only: the result is deterministic.
+#include <cooperative_groups.h>
+
+#include <cstdint>
+#include <cstdlib>
+#include <mutex>
+
+#include "common.cuh"
+#include "launchers.h"
+
+namespace csa2 {
+namespace {
+namespace cg = cooperative_groups;
+
+constexpr int kC = 8;                      // CTAs per row (one cluster)
+constexpr int NT = 512;
+constexpr int NW = NT / 32;
+constexpr int kDigit = 8;
+constexpr int kBins = 1 << kDigit;         // one warp finds the bin: 8 bins per lane
+constexpr int kMaxCand = 4096;
+constexpr int kMaxChunk = 4096;            // keys per CTA
+constexpr int kChunkAlign = 4 * NW;        // chunk = NW segments of a multiple of 4 keys
+static_assert(kC * (kBins / 4) == NT, "one 16-byte histogram store per thread");
+
+struct ClParams {
+  const float* scores;
+  int64_t L;
+  int chunk;                               // keys per CTA, multiple of kChunkAlign
+  int seg;                                 // keys per warp = chunk / NW
+  int count;
+  const int32_t* ids;
+  int32_t* out;
+};
+
+struct Smem {
+  uint32_t keys[kMaxChunk];                // this CTA's keys (0 = not selectable)
+  uint32_t lcand[kMaxChunk];               // this CTA's keys in the threshold bin
+  uint32_t cand[kMaxCand];                 // every CTA's, in CTA order
+  int inbox[2][kC][kBins];                 // histograms stored by each CTA (pass parity)
+  int hist[2][kBins];                      // this CTA's histogram (pass parity)
+  int gsum[kBins];                         // the cluster's histogram
+  uint32_t x_min[kC], x_max[kC];           // stored by each CTA: its selectable keys
+  int x_n[kC];
+  int x_nl[kC], x_above[kC];               // stored by each CTA with its list
+  int x_g[kC], x_e[kC];                    // stored by each CTA: keys above / equal to T
+  int wg[NW], we[NW], wg_off[NW], we_off[NW];
+  uint32_t kmin, kmax;
+  int nsel, nl, above_mine, cnt_g, cnt_e;
+  int bin, above, bin_cnt;
+};
+
+__device__ __forceinline__ uint32_t score_key(float f) {
+  uint32_t u = __float_as_uint(f);
+  if (f != f || u == 0xff800000u) return 0u;       // NaN, -inf: never chosen
+  if (u == 0x80000000u) u = 0u;                    // -0 ranks as +0
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+// Warp 0 only: the bin of h[0..nb) (nb <= kBins) holding the kk-th largest
+// key; sets S.bin, S.above (keys in higher bins) and S.bin_cnt.
+__device__ __forceinline__ void warp_find_bin(const int* h, int nb, int kk, Smem& S) {
+  const int lane = threadIdx.x & 31;
+  int v[8];
+#pragma unroll
+  for (int u = 0; u < 8; ++u) v[u] = 8 * lane + u < nb ? h[8 * lane + u] : 0;
+  const int mine = v[0] + v[1] + v[2] + v[3] + v[4] + v[5] + v[6] + v[7];
+  int x = mine;                              // inclusive suffix sum over the lanes
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_down_sync(0xffffffffu, x, o);
+    if (lane + o < 32) x += y;
+  }
+  int above = x - mine;
+#pragma unroll
+  for (int u = 7; u >= 0; --u) {
+    if (above < kk && above + v[u] >= kk) {
+      S.bin = 8 * lane + u;
+      S.above = above;
+      S.bin_cnt = v[u];
+    }
+    above += v[u];
+  }
+}
+
+__device__ __forceinline__ uint4 keys4(const Smem& S, int i, int lo, int w_hi) {
+  return i < w_hi ? *reinterpret_cast<const uint4*>(&S.keys[i - lo]) : make_uint4(0u, 0u, 0u, 0u);
+}
+
+__device__ __forceinline__ void cluster_arrive() {
+  asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void cluster_wait() {
+  asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+__global__ void __cluster_dims__(kC, 1, 1) __launch_bounds__(NT, 1)
+    topk_cluster_kernel(ClParams p) {
+  extern __shared__ __align__(16) uint8_t smem_raw[];
+  Smem& S = *reinterpret_cast<Smem*>(smem_raw);
+  cg::cluster_group cl = cg::this_cluster();
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int cta = static_cast<int>(cl.block_rank());
+  const int64_t r = blockIdx.x / kC;
+  const int L = static_cast<int>(p.L);
+  const float* s = p.scores + r * p.L;
+  const int lo = min(L, cta * p.chunk), hi = min(L, lo + p.chunk);
+  const int w_lo = lo + warp * p.seg, w_hi = min(hi, w_lo + p.seg);   // empty when w_lo >= hi
+  pdl_wait();                                // the scores come from the kernel before
+  pdl_release();
+
+  if (tid == 0) {
+    S.kmin = 0xffffffffu;
+    S.kmax = 0u;
+    S.nsel = 0;
+    S.nl = 0;
+    S.above_mine = 0;
+    S.cnt_g = 0;
+    S.cnt_e = 0;
+  }
+  S.hist[tid / kBins][tid % kBins] = 0;    // both buffers
+  __syncthreads();
+
+  // ---- this warp's keys; the CTA's smallest / largest selectable key
+  {
+    uint32_t kmin = 0xffffffffu, kmax = 0u;
+    int nsel = 0;
+    const bool vec = (reinterpret_cast<uintptr_t>(s) & 15u) == 0;   // lo, w_lo, i: multiples of 4
+    for (int i = w_lo + 4 * lane; i < w_hi; i += 128) {
+      float f[4];
+      if (vec && i + 3 < w_hi) {
+        const float4 v = __ldg(reinterpret_cast<const float4*>(s + i));
+        f[0] = v.x; f[1] = v.y; f[2] = v.z; f[3] = v.w;
+      } else {
+#pragma unroll
+        for (int u = 0; u < 4; ++u) f[u] = i + u < w_hi ? __ldg(s + i + u) : __int_as_float(0xff800000);
+      }
+      uint32_t k4[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        k4[u] = score_key(f[u]);
+        if (k4[u]) {
+          kmin = min(kmin, k4[u]);
+          kmax = max(kmax, k4[u]);
+          ++nsel;
+        }
+      }
+      *reinterpret_cast<uint4*>(&S.keys[i - lo]) = make_uint4(k4[0], k4[1], k4[2], k4[3]);
+    }
+    kmin = __reduce_min_sync(0xffffffffu, kmin);
+    kmax = __reduce_max_sync(0xffffffffu, kmax);
+    nsel = __reduce_add_sync(0xffffffffu, nsel);
+    if (lane == 0) {
+      atomicMin(&S.kmin, kmin);
+      atomicMax(&S.kmax, kmax);
+      atomicAdd(&S.nsel, nsel);
+    }
+  }
+  __syncthreads();
+  if (tid < kC) {
+    Smem* R = cl.map_shared_rank(&S, tid);
+    R->x_min[cta] = S.kmin;
+    R->x_max[cta] = S.kmax;
+    R->x_n[cta] = S.nsel;
+  }
+  cl.sync();                                 // every CTA's min / max / count is here
+  uint32_t rmin = 0xffffffffu, rmax = 0u;
+  int total_sel = 0, nsel_before = 0;
+#pragma unroll
+  for (int c = 0; c < kC; ++c) {
+    rmin = min(rmin, S.x_min[c]);
+    rmax = max(rmax, S.x_max[c]);
+    total_sel += S.x_n[c];
+    nsel_before += c < cta ? S.x_n[c] : 0;
+  }
+  const bool all = total_sel <= p.count;     // every selectable key is chosen
+
+  // ---- threshold key T, how many keys equal to T to take (take), how many
+  // there are (eqcnt); keys above / equal to T in the CTAs before this one
+  uint32_t T = 0u;
+  int take = 0, eqcnt = 0, cgb = 0, ceb = 0;
+  bool exchange = false;                     // the counts still need an exchange
+  if (all) {
+    cgb = nsel_before;
+    cluster_arrive();
+  } else if (rmin == rmax) {                 // one distinct key, more of it than wanted
+    T = rmin;
+    take = p.count;
+    eqcnt = total_sel;
+    ceb = nsel_before;
+    cluster_arrive();
+  } else {
+    const int common = __clz(rmin ^ rmax);
+    const uint32_t cmask = common == 0 ? 0u : ~0u << (32 - common);
+    uint32_t prefix = rmin & cmask, mask = cmask;
+    int kk = p.count;
+    int lowbit = 32 - common;                // key bits [lowbit-1 : 0] still undecided
+    int par = 0;
+    int my_above = 0;                        // this thread's bins above the threshold bins
+    bool gathered = false;
+    int ncand = 0, my_off = 0;
+    while (lowbit > 0 && !gathered) {
+      const int width = lowbit >= kDigit ? kDigit : lowbit;
+      const int shift = lowbit - width;
+      const uint32_t dmask = (1u << width) - 1u;
+      const int nb = 1 << width;
+      for (int b0 = w_lo; b0 < w_hi; b0 += 128) {
+        const int i = b0 + 4 * lane;
+        const uint4 k4 = keys4(S, i, lo, w_hi);
+        const uint32_t kv[4] = {k4.x, k4.y, k4.z, k4.w};
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+          if (kv[u] && i + u < w_hi && (kv[u] & mask) == prefix)
+            atomicAdd(&S.hist[par][(kv[u] >> shift) & dmask], 1);
+      }
+      __syncthreads();
+      {
+        const int d = tid / (kBins / 4), q4 = 4 * (tid % (kBins / 4));
+        Smem* R = cl.map_shared_rank(&S, d);
+        *reinterpret_cast<int4*>(&R->inbox[par][cta][q4]) = *reinterpret_cast<const int4*>(&S.hist[par][q4]);
+      }
+      cl.sync();                             // every CTA's histogram is here
+      if (tid < nb) {
+        int v = 0;
+#pragma unroll
+        for (int c = 0; c < kC; ++c) v += S.inbox[par][c][tid];
+        S.gsum[tid] = v;
+      }
+      __syncthreads();
+      if (warp == 0) warp_find_bin(S.gsum, nb, kk, S);
+      __syncthreads();
+      const int b = S.bin;
+      if (tid < nb && tid > b) my_above += S.hist[par][tid];
+      kk -= S.above;
+      eqcnt = S.bin_cnt;
+      prefix |= static_cast<uint32_t>(b) << shift;
+      mask |= dmask << shift;
+      lowbit = shift;
+      __syncthreads();                       // every thread has read the histogram
+      if (tid < kBins) S.hist[par][tid] = 0;   // zero again before its next use, two passes on
+      par ^= 1;
+      if (lowbit > 0 && eqcnt <= kMaxCand) {
+        // this CTA's keys in the bin, with how many of its keys lie above it
+        for (int b0 = w_lo; b0 < w_hi; b0 += 128) {
+          const int i = b0 + 4 * lane;
+          const uint4 k4 = keys4(S, i, lo, w_hi);
+          const uint32_t kv[4] = {k4.x, k4.y, k4.z, k4.w};
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const bool m = kv[u] && i + u < w_hi && (kv[u] & mask) == prefix;
+            const unsigned bal = __ballot_sync(0xffffffffu, m);
+            int base = 0;
+            if (lane == 0 && bal) base = atomicAdd(&S.nl, __popc(bal));
+            base = __shfl_sync(0xffffffffu, base, 0);
+            if (m) S.lcand[base + __popc(bal & ((1u << lane) - 1u))] = kv[u];
+          }
+        }
+        const int a = __reduce_add_sync(0xffffffffu, my_above);
+        if (lane == 0 && a) atomicAdd(&S.above_mine, a);
+        __syncthreads();
+        if (tid < kC) {
+          Smem* R = cl.map_shared_rank(&S, tid);
+          R->x_nl[cta] = S.nl;
+          R->x_above[cta] = S.above_mine;
+        }
+        cl.sync();                           // every CTA's list and count is here
+        int off[kC];
+        int acc = 0;
+#pragma unroll
+        for (int c = 0; c < kC; ++c) {
+          off[c] = acc;
+          if (c == cta) my_off = acc;
+          acc += S.x_nl[c];
+          cgb += c < cta ? S.x_above[c] : 0;
+        }
+        ncand = acc;                         // == eqcnt
+        for (int j = tid; j < ncand; j += NT) {
+          int c = 0, base = 0;               // the last CTA whose list starts at or before j
+#pragma unroll
+          for (int u = 1; u < kC; ++u)
+            if (j >= off[u]) {
+              c = u;
+              base = off[u];
+            }
+          S.cand[j] = cl.map_shared_rank(S.lcand, c)[j - base];
+        }
+        gathered = true;
+        __syncthreads();
+        cluster_arrive();                    // this CTA reads no other CTA's memory from here on
+      }
+    }
+    if (gathered) {
+      // further passes over the candidates alone (both histograms are zero)
+      int lp = 0;
+      while (lowbit > 0) {
+        const int width = lowbit >= kDigit ? kDigit : lowbit;
+        const int shift = lowbit - width;
+        const uint32_t dmask = (1u << width) - 1u;
+        for (int j = tid; j < ncand; j += NT) {
+          const uint32_t key = S.cand[j];
+          if ((key & mask) == prefix) atomicAdd(&S.hist[lp][(key >> shift) & dmask], 1);
+        }
+        __syncthreads();
+        if (warp == 0) warp_find_bin(S.hist[lp], 1 << width, kk, S);
+        __syncthreads();
+        prefix |= static_cast<uint32_t>(S.bin) << shift;
+        mask |= dmask << shift;
+        kk -= S.above;
+        eqcnt = S.bin_cnt;
+        lowbit = shift;
+        // zero for the pass after next, whose counts start after the next
+        // pass's first barrier
+        if (tid < kBins) S.hist[lp][tid] = 0;
+        lp ^= 1;
+      }
+      T = prefix;
+      take = kk;
+      // candidates above / equal to T listed before this CTA's own
+      int g = 0, e = 0;
+      for (int j = tid; j < my_off; j += NT) {
+        const uint32_t key = S.cand[j];
+        g += key > T;
+        e += key == T;
+      }
+      g = __reduce_add_sync(0xffffffffu, g);
+      e = __reduce_add_sync(0xffffffffu, e);
+      if (lane == 0 && (g | e)) {
+        atomicAdd(&S.cnt_g, g);
+        atomicAdd(&S.cnt_e, e);
+      }
+      __syncthreads();
+      cgb += S.cnt_g;
+      ceb = S.cnt_e;
+    } else {
+      // the bin never fit the list: every key bit is decided, counts follow below
+      T = prefix;
+      take = kk;
+      exchange = true;
+    }
+  }
+
+  // ---- per warp: keys above / equal to T.  All keys equal to T taken (the
+  // usual case): one sweep compacts each warp's picks, in order, into its own
+  // part of the key buffer (never past the keys it has read).
+  const bool simple = all || take >= eqcnt;
+  const uint32_t thr = all ? 1u : T;
+  const unsigned lt = (1u << lane) - 1u;
+  {
+    int g = 0, e = 0;
+    if (simple) {
+      for (int b0 = w_lo; b0 < w_hi; b0 += 128) {
+        const int i = b0 + 4 * lane;
+        const uint4 k4 = keys4(S, i, lo, w_hi);
+        const uint32_t kv[4] = {k4.x, k4.y, k4.z, k4.w};
+        int sel_m = 0;
+#pragma unroll
+        for (int u = 0; u < 4; ++u) sel_m |= (kv[u] >= thr && i + u < w_hi) << u;
+        if (!__any_sync(0xffffffffu, sel_m)) continue;
+        int lower = 0, total = 0;
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const unsigned sb = __ballot_sync(0xffffffffu, (sel_m >> u) & 1);
+          lower += __popc(sb & lt);
+          total += __popc(sb);
+        }
+        int q = g + lower;
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+          if ((sel_m >> u) & 1) S.keys[w_lo - lo + q++] = static_cast<uint32_t>(i + u);
+        g += total;
+      }
+    } else {
+      for (int b0 = w_lo; b0 < w_hi; b0 += 128) {
+        const int i = b0 + 4 * lane;
+        const uint4 k4 = keys4(S, i, lo, w_hi);
+        const uint32_t kv[4] = {k4.x, k4.y, k4.z, k4.w};
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const bool valid = kv[u] != 0u && i + u < w_hi;
+          g += (valid && kv[u] > T) ? 1 : 0;
+          e += (valid && kv[u] == T) ? 1 : 0;
+        }
+      }
+      g = __reduce_add_sync(0xffffffffu, g);
+      e = __reduce_add_sync(0xffffffffu, e);
+    }
+    if (lane == 0) {
+      S.wg[warp] = g;
+      S.we[warp] = e;
+    }
+  }
+  __syncthreads();
+  if (warp == 0) {
+    const int g = lane < NW ? S.wg[lane] : 0, e = lane < NW ? S.we[lane] : 0;
+    int gi = g, ei = e;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int yg = __shfl_up_sync(0xffffffffu, gi, o), ye = __shfl_up_sync(0xffffffffu, ei, o);
+      if (lane >= o) {
+        gi += yg;
+        ei += ye;
+      }
+    }
+    if (lane < NW) {
+      S.wg_off[lane] = gi - g;
+      S.we_off[lane] = ei - e;
+    }
+    const int gt = __shfl_sync(0xffffffffu, gi, 31), et = __shfl_sync(0xffffffffu, ei, 31);
+    if (exchange && lane < kC) {             // this CTA's totals to every CTA
+      Smem* R = cl.map_shared_rank(&S, lane);
+      R->x_g[cta] = gt;
+      R->x_e[cta] = et;
+    }
+  }
+  if (exchange) {
+    cl.sync();                               // every CTA's counts are here
+#pragma unroll
+    for (int c = 0; c < kC; ++c) {
+      cgb += c < cta ? S.x_g[c] : 0;
+      ceb += c < cta ? S.x_e[c] : 0;
+    }
+    cluster_arrive();
+  } else {
+    __syncthreads();
+  }
+
+  int32_t* o = p.out + r * static_cast<int64_t>(p.count);
+  const int g_before = cgb + S.wg_off[warp];
+  const int e_before = ceb + S.we_off[warp];
+  if (simple) {
+    const int sel_start = g_before + min(e_before, take);
+    for (int j = lane; j < S.wg[warp]; j += 32) {
+      const int q = sel_start + j;
+      const int posn = static_cast<int>(S.keys[w_lo - lo + j]);
+      if (q < p.count) o[q] = p.ids ? p.ids[r * p.L + posn] : posn;
+    }
+  } else {
+    int run_sel = g_before + min(e_before, take), run_eq = e_before;
+    for (int b0 = w_lo; b0 < w_hi; b0 += 128) {
+      const int i = b0 + 4 * lane;
+      const uint4 k4 = keys4(S, i, lo, w_hi);
+      const uint32_t kv[4] = {k4.x, k4.y, k4.z, k4.w};
+      int sel_m = 0, eq_m = 0;
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const bool valid = kv[u] != 0u && i + u < w_hi;
+        sel_m |= (valid && kv[u] > T) << u;
+        eq_m |= (valid && kv[u] == T) << u;
+      }
+      // position order is lane-major: lower lanes' keys, then this lane's
+      // earlier keys, come first
+      int eq_lower = 0, warp_eq = 0;
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const unsigned eb = __ballot_sync(0xffffffffu, (eq_m >> u) & 1);
+        eq_lower += __popc(eb & lt);
+        warp_eq += __popc(eb);
+      }
+      int rank = run_eq + eq_lower;
+#pragma unroll
+      for (int u = 0; u < 4; ++u)
+        if ((eq_m >> u) & 1) {
+          if (rank < take) sel_m |= 1 << u;
+          ++rank;
+        }
+      int sel_lower = 0, warp_sel = 0;
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const unsigned sb = __ballot_sync(0xffffffffu, (sel_m >> u) & 1);
+        sel_lower += __popc(sb & lt);
+        warp_sel += __popc(sb);
+      }
+      int pos = run_sel + sel_lower;
+#pragma unroll
+      for (int u = 0; u < 4; ++u)
+        if ((sel_m >> u) & 1) {
+          if (pos < p.count) o[pos] = p.ids ? p.ids[r * p.L + i + u] : i + u;
+          ++pos;
+        }
+      run_sel += warp_sel;
+      run_eq += warp_eq;
+    }
+  }
+  // padding: positions beyond the selectable keys
+  const int n_out = all ? total_sel : p.count;
+  for (int q = n_out + cta * NT + tid; q < p.count; q += kC * NT) o[q] = -1;
+  // no CTA leaves while another may still read its shared memory
+  cluster_wait();
+}
+
+}  // namespace
+
+bool select_topk_cluster_applies(int64_t rows, int64_t L, int count0, int count1) {
+  return count1 <= 0 && count0 > 0 && rows > 0 && rows < sm_count() && L > 0 &&
+         L <= static_cast<int64_t>(kC) * kMaxChunk && !getenv("CSA2_TOPK_NO_CLUSTER");
+}
+
+csa2_status launch_select_topk_cluster(const float* scores, int64_t rows, int64_t L, int count,
+                                       const int32_t* ids, int32_t* out, cudaStream_t stream) {
+  if (!select_topk_cluster_applies(rows, L, count, 0)) return CSA2_ERR_UNSUPPORTED;
+  ClParams p;
+  p.scores = scores;
+  p.L = L;
+  const int64_t per = (L + kC - 1) / kC;
+  p.chunk = static_cast<int>((per + kChunkAlign - 1) / kChunkAlign * kChunkAlign);
+  p.seg = p.chunk / NW;
+  p.count = count;
+  p.ids = ids;
+  p.out = out;
+  static std::once_flag once;
+  static cudaError_t attr = cudaSuccess;
+  std::call_once(once, [] {
+    attr = cudaFuncSetAttribute(topk_cluster_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                static_cast<int>(sizeof(Smem)));
+  });
+  if (attr != cudaSuccess) return fail(CSA2_ERR_CUDA, "select_topk_cluster: shared-memory opt-in failed");
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(rows * kC));
+  cfg.blockDim = dim3(NT);
+  cfg.dynamicSmemBytes = sizeof(Smem);
+  cfg.stream = stream;
+  cudaLaunchAttribute at[1] = {pdl_attribute()};
+  cfg.attrs = at;
+  cfg.numAttrs = 1;
+  begin_launch(stream);
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, topk_cluster_kernel, p);
+  note_launch(LK_TOPK, 1, stream);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return fail(CSA2_ERR_CUDA, "select_topk_cluster: launch failed: %s", cudaGetErrorString(e));
+  }
+  return check_launch("select_topk_cluster");
+}
+
+}  // namespace csa2

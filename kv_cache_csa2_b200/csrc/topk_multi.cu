@@ -665,6 +665,8 @@ size_t select_topk_multi_workspace(int64_t rows, int64_t L, int) {
 csa2_status launch_select_topk2(const float* scores, int64_t rows, int64_t L, int count0,
                                 const int32_t* ids, int32_t* out0, int count1, int32_t* out1,
                                 void* ws, size_t ws_bytes, cudaStream_t stream, bool ws_cleared) {
+  if (select_topk_cluster_applies(rows, L, count0, count1))
+    return launch_select_topk_cluster(scores, rows, L, count0, ids, out0, stream);
   if (cta_kernel_takes(rows, L))
     return launch_select_topk_cta(scores, rows, L, count0, ids, out0, count1, out1, stream);
   if (!multi_applies(rows, L)) return CSA2_ERR_UNSUPPORTED;

@@ -173,6 +173,8 @@ def test_index_scores_pool_parity(B, Q, H, d, N, P):
 def _score_rows(r, rows, L, kind):
     if kind == "ties":
         s = r.integers(-20, 20, (rows, L)).astype(np.float32)
+    elif kind == "dense_ties":      # the threshold bin keeps most of the row in every pass
+        s = np.where(r.random((rows, L)) < 0.8, np.float32(1.0), np.float32(2.0)).astype(np.float32)
     else:
         s = r.standard_normal((rows, L)).astype(np.float32)
     s[r.random((rows, L)) < 0.05] = -np.inf
@@ -182,8 +184,9 @@ def _score_rows(r, rows, L, kind):
 
 @pytest.mark.parametrize("rows,L,count", [(5, 1000, 37), (3, 4096, 2048), (2, 300, 1000), (1, 1, 1),
                                           (8, 16384, 2048), (2, 32768, 16384), (3, 20001, 5000),
-                                          (4, 70000, 2048), (2, 262144, 16384), (64, 2000, 256)])
-@pytest.mark.parametrize("kind", ["normal", "ties"])
+                                          (4, 70000, 2048), (2, 262144, 16384), (64, 2000, 256),
+                                          (200, 3000, 100), (5, 32765, 7000)])
+@pytest.mark.parametrize("kind", ["normal", "ties", "dense_ties"])
 def test_select_topk_exact(rows, L, count, kind):
     r = _rng(7)
     s = _score_rows(r, rows, L, kind)
@@ -193,13 +196,46 @@ def test_select_topk_exact(rows, L, count, kind):
     assert np.array_equal(got, want)
 
 
-@pytest.mark.parametrize("rows,L,count", [(3, 4096, 2048), (8, 16384, 2048), (2, 32768, 16384)])
-def test_select_topk_chunked_path(rows, L, count, monkeypatch):
-    """Rows up to 32768 scores normally take the one-CTA kernel; the
-    cooperative kernel's one-chunk path gives the same result."""
-    monkeypatch.setenv("CSA2_TOPK_NO_CTA", "1")
+@pytest.mark.parametrize("rows,L,count", [(3, 4096, 2048), (8, 16384, 2048), (2, 32768, 16384),
+                                          (3, 20001, 5000)])
+@pytest.mark.parametrize("path", ["one_cta", "chunked"])
+@pytest.mark.parametrize("kind", ["ties", "dense_ties"])
+def test_select_topk_short_row_paths(rows, L, count, path, kind, monkeypatch):
+    """Short rows of a small batch normally take the 8-CTA cluster kernel;
+    the one-CTA kernel and the cooperative kernel's one-chunk path give the
+    same result."""
+    monkeypatch.setenv("CSA2_TOPK_NO_CLUSTER", "1")
+    if path == "chunked":
+        monkeypatch.setenv("CSA2_TOPK_NO_CTA", "1")
     r = _rng(17)
-    s = _score_rows(r, rows, L, "ties")
+    s = _score_rows(r, rows, L, kind)
+    got = K.csa2_select_topk(U.dev(s), count).cpu().numpy()
+    want = O.select_top(np.where(np.isnan(s), -np.inf, s).astype(np.float64), count)
+    assert np.array_equal(got, want)
+
+
+@pytest.mark.parametrize("case", ["all_equal", "nothing_selectable", "few_selectable", "one_key",
+                                  "narrow_band", "odd_rows"])
+def test_select_topk_cluster_edges(case):
+    """Edge rows of the cluster kernel (8 rows, at most 32768 scores)."""
+    r = _rng(19)
+    rows, L, count = 8, 16384, 2048
+    if case == "all_equal":
+        s = np.full((rows, L), 0.5, dtype=np.float32)
+    elif case == "nothing_selectable":
+        s = np.where(r.random((rows, L)) < 0.5, np.float32(-np.inf), np.float32(np.nan)).astype(np.float32)
+    elif case == "few_selectable":       # fewer selectable scores than count: -1 padding
+        s = np.full((rows, L), -np.inf, dtype=np.float32)
+        s[r.random((rows, L)) < 0.05] = 3.0
+        s[:, 5] = 4.0
+    elif case == "one_key":
+        rows, L, count = 3, 1, 1
+        s = r.standard_normal((rows, L)).astype(np.float32)
+    elif case == "narrow_band":          # long common key prefix, many near-ties
+        s = (1.0 + 1e-6 * r.integers(0, 50, (rows, L))).astype(np.float32)
+    else:                                # row starts off 16 bytes: unvectorised loads
+        rows, L, count = 5, 4099, 1000
+        s = r.standard_normal((rows, L)).astype(np.float32)
     got = K.csa2_select_topk(U.dev(s), count).cpu().numpy()
     want = O.select_top(np.where(np.isnan(s), -np.inf, s).astype(np.float64), count)
     assert np.array_equal(got, want)
