@@ -45,10 +45,13 @@ csa2_status launch_select_topk_cta(const float* scores, int64_t rows, int64_t L,
                                    const int32_t* ids, int32_t* out0, int count1, int32_t* out1,
                                    cudaStream_t stream);
 // A cluster of 8 CTAs per row, no workspace: one selection (count1 <= 0) of
-// rows of up to 32768 scores when there are fewer rows than SMs.
+// rows of up to 262144 scores when there are fewer rows than SMs.  With
+// `gather`, key i of row r is scores[r * src_stride + gather[r * L + i]]
+// (negative entries are not selectable).
 bool select_topk_cluster_applies(int64_t rows, int64_t L, int count0, int count1);
 csa2_status launch_select_topk_cluster(const float* scores, int64_t rows, int64_t L, int count,
-                                       const int32_t* ids, int32_t* out, cudaStream_t stream);
+                                       const int32_t* ids, int32_t* out, cudaStream_t stream,
+                                       const int32_t* gather = nullptr, int64_t src_stride = 0);
 csa2_status launch_select_topk(const float* scores, int64_t rows, int64_t L, int count,
                                const int32_t* ids, int32_t* out, void* ws, size_t ws_bytes,
                                cudaStream_t stream);

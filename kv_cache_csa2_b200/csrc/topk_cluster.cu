@@ -1,9 +1,11 @@
-// Top-k selection of short rows (up to 32768 scores) with a cluster of 8 CTAs
-// per row, for batches too small to fill the GPU with one CTA per row (the
-// hierarchical indexer's pool in a Reindex layer: 8 rows of 16384).  Sources:
-// "读完这篇，你就搞懂 DeepSeek v4 了", 闪电索引机制 (keep the k best
-// entries); "Recall之王", Hierarchical Sparse Indexer (the Reindex layer's
-// top-k inside the pool).
+// Top-k selection with a cluster of 8 CTAs per row, for batches too small to
+// fill the GPU with one CTA per row: the hierarchical indexer's pool in a
+// Reindex layer (8 rows of 16384) and a Full layer's pool and top-k (8 rows
+// of 262144).  Two variants: 512 threads and up to 4096 keys per CTA (rows of
+// up to 32768), 1024 threads and up to 32768 keys per CTA (rows of up to
+// 262144).  Sources: "读完这篇，你就搞懂 DeepSeek v4 了", 闪电索引机制
+// (keep the k best entries); "Recall之王", Hierarchical Sparse Indexer (the
+// Full layer's pool and its top-k; the Reindex layer's top-k inside the pool).
 //
 // Same result as the one-CTA kernel: score descending, ties to the lower
 // position, -inf and NaN never chosen, -0 ranks as +0; selected positions
@@ -38,28 +40,30 @@ namespace {
 namespace cg = cooperative_groups;
 
 constexpr int kC = 8;                      // CTAs per row (one cluster)
-constexpr int NT = 512;
-constexpr int NW = NT / 32;
 constexpr int kDigit = 8;
 constexpr int kBins = 1 << kDigit;         // one warp finds the bin: 8 bins per lane
 constexpr int kMaxCand = 4096;
-constexpr int kMaxChunk = 4096;            // keys per CTA
-constexpr int kChunkAlign = 4 * NW;        // chunk = NW segments of a multiple of 4 keys
-static_assert(kC * (kBins / 4) == NT, "one 16-byte histogram store per thread");
+constexpr int kHistStores = kC * (kBins / 4);   // 16-byte histogram stores per CTA and pass
 
 struct ClParams {
   const float* scores;
   int64_t L;
-  int chunk;                               // keys per CTA, multiple of kChunkAlign
-  int seg;                                 // keys per warp = chunk / NW
+  int chunk;                               // keys per CTA, multiple of 4 * warps
+  int seg;                                 // keys per warp = chunk / warps
   int count;
   const int32_t* ids;
   int32_t* out;
+  // when set, key i of row r is scores[r * src_stride + gather[r * L + i]]
+  // (a negative entry: not selectable)
+  const int32_t* gather;
+  int64_t src_stride;
 };
 
+template <int NT, int MAXCHUNK>
 struct Smem {
-  uint32_t keys[kMaxChunk];                // this CTA's keys (0 = not selectable)
-  uint32_t lcand[kMaxChunk];               // this CTA's keys in the threshold bin
+  static constexpr int NW = NT / 32;
+  uint32_t keys[MAXCHUNK];                 // this CTA's keys (0 = not selectable)
+  uint32_t lcand[kMaxCand];                // this CTA's keys in the threshold bin
   uint32_t cand[kMaxCand];                 // every CTA's, in CTA order
   int inbox[2][kC][kBins];                 // histograms stored by each CTA (pass parity)
   int hist[2][kBins];                      // this CTA's histogram (pass parity)
@@ -83,7 +87,8 @@ __device__ __forceinline__ uint32_t score_key(float f) {
 
 // Warp 0 only: the bin of h[0..nb) (nb <= kBins) holding the kk-th largest
 // key; sets S.bin, S.above (keys in higher bins) and S.bin_cnt.
-__device__ __forceinline__ void warp_find_bin(const int* h, int nb, int kk, Smem& S) {
+template <class SM>
+__device__ __forceinline__ void warp_find_bin(const int* h, int nb, int kk, SM& S) {
   const int lane = threadIdx.x & 31;
   int v[8];
 #pragma unroll
@@ -107,7 +112,8 @@ __device__ __forceinline__ void warp_find_bin(const int* h, int nb, int kk, Smem
   }
 }
 
-__device__ __forceinline__ uint4 keys4(const Smem& S, int i, int lo, int w_hi) {
+template <class SM>
+__device__ __forceinline__ uint4 keys4(const SM& S, int i, int lo, int w_hi) {
   return i < w_hi ? *reinterpret_cast<const uint4*>(&S.keys[i - lo]) : make_uint4(0u, 0u, 0u, 0u);
 }
 
@@ -118,10 +124,13 @@ __device__ __forceinline__ void cluster_wait() {
   asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
 
+template <int NT, int MAXCHUNK>
 __global__ void __cluster_dims__(kC, 1, 1) __launch_bounds__(NT, 1)
     topk_cluster_kernel(ClParams p) {
+  using SM = Smem<NT, MAXCHUNK>;
+  constexpr int NW = SM::NW;
   extern __shared__ __align__(16) uint8_t smem_raw[];
-  Smem& S = *reinterpret_cast<Smem*>(smem_raw);
+  SM& S = *reinterpret_cast<SM*>(smem_raw);
   cg::cluster_group cl = cg::this_cluster();
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int cta = static_cast<int>(cl.block_rank());
@@ -142,7 +151,7 @@ __global__ void __cluster_dims__(kC, 1, 1) __launch_bounds__(NT, 1)
     S.cnt_g = 0;
     S.cnt_e = 0;
   }
-  S.hist[tid / kBins][tid % kBins] = 0;    // both buffers
+  for (int i = tid; i < 2 * kBins; i += NT) (&S.hist[0][0])[i] = 0;   // both buffers
   __syncthreads();
 
   // ---- this warp's keys; the CTA's smallest / largest selectable key
@@ -150,9 +159,17 @@ __global__ void __cluster_dims__(kC, 1, 1) __launch_bounds__(NT, 1)
     uint32_t kmin = 0xffffffffu, kmax = 0u;
     int nsel = 0;
     const bool vec = (reinterpret_cast<uintptr_t>(s) & 15u) == 0;   // lo, w_lo, i: multiples of 4
+    const int32_t* gidx = p.gather ? p.gather + r * p.L : nullptr;
+    const float* src = p.scores + r * p.src_stride;
     for (int i = w_lo + 4 * lane; i < w_hi; i += 128) {
       float f[4];
-      if (vec && i + 3 < w_hi) {
+      if (gidx) {
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int g = i + u < w_hi ? __ldg(gidx + i + u) : -1;
+          f[u] = g >= 0 && g < p.src_stride ? __ldg(src + g) : __int_as_float(0xff800000);
+        }
+      } else if (vec && i + 3 < w_hi) {
         const float4 v = __ldg(reinterpret_cast<const float4*>(s + i));
         f[0] = v.x; f[1] = v.y; f[2] = v.z; f[3] = v.w;
       } else {
@@ -182,7 +199,7 @@ __global__ void __cluster_dims__(kC, 1, 1) __launch_bounds__(NT, 1)
   }
   __syncthreads();
   if (tid < kC) {
-    Smem* R = cl.map_shared_rank(&S, tid);
+    SM* R = cl.map_shared_rank(&S, tid);
     R->x_min[cta] = S.kmin;
     R->x_max[cta] = S.kmax;
     R->x_n[cta] = S.nsel;
@@ -238,9 +255,9 @@ __global__ void __cluster_dims__(kC, 1, 1) __launch_bounds__(NT, 1)
             atomicAdd(&S.hist[par][(kv[u] >> shift) & dmask], 1);
       }
       __syncthreads();
-      {
+      if (tid < kHistStores) {
         const int d = tid / (kBins / 4), q4 = 4 * (tid % (kBins / 4));
-        Smem* R = cl.map_shared_rank(&S, d);
+        SM* R = cl.map_shared_rank(&S, d);
         *reinterpret_cast<int4*>(&R->inbox[par][cta][q4]) = *reinterpret_cast<const int4*>(&S.hist[par][q4]);
       }
       cl.sync();                             // every CTA's histogram is here
@@ -283,7 +300,7 @@ __global__ void __cluster_dims__(kC, 1, 1) __launch_bounds__(NT, 1)
         if (lane == 0 && a) atomicAdd(&S.above_mine, a);
         __syncthreads();
         if (tid < kC) {
-          Smem* R = cl.map_shared_rank(&S, tid);
+          SM* R = cl.map_shared_rank(&S, tid);
           R->x_nl[cta] = S.nl;
           R->x_above[cta] = S.above_mine;
         }
@@ -431,7 +448,7 @@ __global__ void __cluster_dims__(kC, 1, 1) __launch_bounds__(NT, 1)
     }
     const int gt = __shfl_sync(0xffffffffu, gi, 31), et = __shfl_sync(0xffffffffu, ei, 31);
     if (exchange && lane < kC) {             // this CTA's totals to every CTA
-      Smem* R = cl.map_shared_rank(&S, lane);
+      SM* R = cl.map_shared_rank(&S, lane);
       R->x_g[cta] = gt;
       R->x_e[cta] = et;
     }
@@ -512,48 +529,65 @@ __global__ void __cluster_dims__(kC, 1, 1) __launch_bounds__(NT, 1)
   cluster_wait();
 }
 
-}  // namespace
+constexpr int kSmallThreads = 512, kSmallChunk = 4096;
+constexpr int kLargeThreads = 1024, kLargeChunk = 32768;
+static_assert(kHistStores <= kSmallThreads, "one 16-byte histogram store per thread");
 
-bool select_topk_cluster_applies(int64_t rows, int64_t L, int count0, int count1) {
-  return count1 <= 0 && count0 > 0 && rows > 0 && rows < sm_count() && L > 0 &&
-         L <= static_cast<int64_t>(kC) * kMaxChunk && !getenv("CSA2_TOPK_NO_CLUSTER");
-}
-
-csa2_status launch_select_topk_cluster(const float* scores, int64_t rows, int64_t L, int count,
-                                       const int32_t* ids, int32_t* out, cudaStream_t stream) {
-  if (!select_topk_cluster_applies(rows, L, count, 0)) return CSA2_ERR_UNSUPPORTED;
-  ClParams p;
-  p.scores = scores;
-  p.L = L;
-  const int64_t per = (L + kC - 1) / kC;
-  p.chunk = static_cast<int>((per + kChunkAlign - 1) / kChunkAlign * kChunkAlign);
+template <int NT, int MAXCHUNK>
+csa2_status launch_variant(ClParams p, int64_t rows, cudaStream_t stream) {
+  constexpr int NW = NT / 32;
+  const int64_t per = (p.L + kC - 1) / kC;
+  p.chunk = static_cast<int>((per + 4 * NW - 1) / (4 * NW) * (4 * NW));
   p.seg = p.chunk / NW;
-  p.count = count;
-  p.ids = ids;
-  p.out = out;
+  if (p.chunk > MAXCHUNK) return CSA2_ERR_UNSUPPORTED;
+  using SM = Smem<NT, MAXCHUNK>;
   static std::once_flag once;
   static cudaError_t attr = cudaSuccess;
   std::call_once(once, [] {
-    attr = cudaFuncSetAttribute(topk_cluster_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                static_cast<int>(sizeof(Smem)));
+    attr = cudaFuncSetAttribute(topk_cluster_kernel<NT, MAXCHUNK>,
+                                cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(sizeof(SM)));
   });
   if (attr != cudaSuccess) return fail(CSA2_ERR_CUDA, "select_topk_cluster: shared-memory opt-in failed");
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(rows * kC));
   cfg.blockDim = dim3(NT);
-  cfg.dynamicSmemBytes = sizeof(Smem);
+  cfg.dynamicSmemBytes = sizeof(SM);
   cfg.stream = stream;
   cudaLaunchAttribute at[1] = {pdl_attribute()};
   cfg.attrs = at;
   cfg.numAttrs = 1;
   begin_launch(stream);
-  const cudaError_t e = cudaLaunchKernelEx(&cfg, topk_cluster_kernel, p);
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, topk_cluster_kernel<NT, MAXCHUNK>, p);
   note_launch(LK_TOPK, 1, stream);
   if (e != cudaSuccess) {
     cudaGetLastError();
     return fail(CSA2_ERR_CUDA, "select_topk_cluster: launch failed: %s", cudaGetErrorString(e));
   }
   return check_launch("select_topk_cluster");
+}
+
+}  // namespace
+
+bool select_topk_cluster_applies(int64_t rows, int64_t L, int count0, int count1) {
+  return count1 <= 0 && count0 > 0 && rows > 0 && rows < sm_count() && L > 0 &&
+         L <= static_cast<int64_t>(kC) * kLargeChunk && !getenv("CSA2_TOPK_NO_CLUSTER");
+}
+
+csa2_status launch_select_topk_cluster(const float* scores, int64_t rows, int64_t L, int count,
+                                       const int32_t* ids, int32_t* out, cudaStream_t stream,
+                                       const int32_t* gather, int64_t src_stride) {
+  if (!select_topk_cluster_applies(rows, L, count, 0)) return CSA2_ERR_UNSUPPORTED;
+  ClParams p;
+  p.scores = scores;
+  p.L = L;
+  p.count = count;
+  p.ids = ids;
+  p.out = out;
+  p.gather = gather;
+  p.src_stride = gather ? src_stride : L;
+  if (L <= static_cast<int64_t>(kC) * kSmallChunk)
+    return launch_variant<kSmallThreads, kSmallChunk>(p, rows, stream);
+  return launch_variant<kLargeThreads, kLargeChunk>(p, rows, stream);
 }
 
 }  // namespace csa2

@@ -667,6 +667,17 @@ csa2_status launch_select_topk2(const float* scores, int64_t rows, int64_t L, in
                                 void* ws, size_t ws_bytes, cudaStream_t stream, bool ws_cleared) {
   if (select_topk_cluster_applies(rows, L, count0, count1))
     return launch_select_topk_cluster(scores, rows, L, count0, ids, out0, stream);
+  if (count0 > 0 && count1 > 0 && !ids &&
+      select_topk_cluster_applies(rows, L, std::max(count0, count1), 0)) {
+    // The smaller selection lies inside the larger one (same order, same tie
+    // rule), so it runs over the larger one's positions: pool, then top-k.
+    const bool first_big = count0 >= count1;
+    const int big = first_big ? count0 : count1, small = first_big ? count1 : count0;
+    int32_t* out_big = first_big ? out0 : out1;
+    int32_t* out_small = first_big ? out1 : out0;
+    CSA2_TRY(launch_select_topk_cluster(scores, rows, L, big, nullptr, out_big, stream));
+    return launch_select_topk_cluster(scores, rows, big, small, out_big, out_small, stream, out_big, L);
+  }
   if (cta_kernel_takes(rows, L))
     return launch_select_topk_cta(scores, rows, L, count0, ids, out0, count1, out1, stream);
   if (!multi_applies(rows, L)) return CSA2_ERR_UNSUPPORTED;

@@ -251,6 +251,28 @@ def test_select_topk_signed_zero_ties(L):
     assert np.array_equal(got, O.select_top(s.astype(np.float64), L // 2))
 
 
+@pytest.mark.parametrize("B,Q,H,d,N,k_top,P", [(2, 3, 16, 64, 5000, 300, 1000),
+                                              (2, 2, 2, 32, 5000, 300, 4500),
+                                              (3, 1, 8, 32, 70000, 100, 3000),
+                                              (8, 1, 64, 128, 262144, 2048, 16384)])
+@pytest.mark.parametrize("path", ["cluster", "multi"])
+def test_index_topk_full_pool_and_topk(B, Q, H, d, N, k_top, P, path, monkeypatch):
+    """A Full layer's two selections (the pool and the top-k) against the
+    oracle's selection over the same scores (the scoring kernel is
+    deterministic).  The cluster path selects the pool, then the top-k inside
+    it; the cooperative kernel selects both in the same passes.  H = 2 leaves
+    many scores at exactly 0 (ReLU), so ties reach into the pool."""
+    if path == "multi":
+        monkeypatch.setenv("CSA2_TOPK_NO_CLUSTER", "1")
+    r = _rng(21)
+    q, w, k = _index_inputs(r, B, Q, H, d, N)
+    dq, dw, dk = U.dev_bf16(q), U.dev(w), U.dev_bf16(k)
+    topk, pool = K.csa2_index_topk(K.FULL, dq, dw, dk, k_top, pool_size=P)
+    s = K.csa2_index_scores(dq, dw, dk).cpu().numpy().astype(np.float64)
+    assert np.array_equal(pool.cpu().numpy(), O.select_top(s, P))
+    assert np.array_equal(topk.cpu().numpy(), O.select_top(s, k_top))
+
+
 def test_select_topk_maps_ids():
     r = _rng(8)
     s = _score_rows(r, 4, 3000, "ties")
