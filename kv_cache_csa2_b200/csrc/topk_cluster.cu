@@ -59,14 +59,23 @@ struct ClParams {
   int64_t src_stride;
 };
 
-template <int NT, int MAXCHUNK>
+template <int NT, int MAXCHUNK, int SURV>
 struct Smem {
   static constexpr int NW = NT / 32;
   uint32_t keys[MAXCHUNK];                 // this CTA's keys (0 = not selectable)
   uint32_t lcand[kMaxCand];                // this CTA's keys in the threshold bin
-  uint32_t cand[kMaxCand];                 // every CTA's, in CTA order
-  int inbox[2][kC][kBins];                 // histograms stored by each CTA (pass parity)
-  int hist[2][kBins];                      // this CTA's histogram (pass parity)
+  union {
+    int inbox[2][kC][kBins];               // histograms stored by each CTA (pass parity)
+    uint32_t cand[kMaxCand];               // after the passes: every CTA's list, in CTA order
+  } x;
+  union {
+    int whist[NW][kBins];                  // each warp's histogram of the pass
+    struct {                               // after the passes: keys in or above the
+      uint32_t key[SURV];                  // threshold bin, in position order, with
+      uint16_t pos[SURV];                  // their positions in the chunk
+    } surv;
+  } w;
+  int hist[2][kBins];                      // the CTA's histogram; the local passes' (parity)
   int gsum[kBins];                         // the cluster's histogram
   uint32_t x_min[kC], x_max[kC];           // stored by each CTA: its selectable keys
   int x_n[kC];
@@ -74,9 +83,10 @@ struct Smem {
   int x_g[kC], x_e[kC];                    // stored by each CTA: keys above / equal to T
   int wg[NW], we[NW], wg_off[NW], we_off[NW];
   uint32_t kmin, kmax;
-  int nsel, nl, above_mine, cnt_g, cnt_e;
+  int nsel, nl, cnt_g, cnt_e;
   int bin, above, bin_cnt;
 };
+static_assert(sizeof(uint32_t) * kMaxCand <= sizeof(int) * 2 * kC * kBins, "list fits the inboxes");
 
 __device__ __forceinline__ uint32_t score_key(float f) {
   uint32_t u = __float_as_uint(f);
@@ -124,10 +134,33 @@ __device__ __forceinline__ void cluster_wait() {
   asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
 
-template <int NT, int MAXCHUNK>
+// Exclusive prefix over the warps of per-warp counts (g, e) in S.wg / S.we
+// (warp 0 computes it into S.wg_off / S.we_off and returns the CTA totals).
+template <class SM, int NW>
+__device__ __forceinline__ void warp_offsets(SM& S, int* g_tot, int* e_tot) {
+  const int lane = threadIdx.x & 31;
+  const int g = lane < NW ? S.wg[lane] : 0, e = lane < NW ? S.we[lane] : 0;
+  int gi = g, ei = e;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int yg = __shfl_up_sync(0xffffffffu, gi, o), ye = __shfl_up_sync(0xffffffffu, ei, o);
+    if (lane >= o) {
+      gi += yg;
+      ei += ye;
+    }
+  }
+  if (lane < NW) {
+    S.wg_off[lane] = gi - g;
+    S.we_off[lane] = ei - e;
+  }
+  *g_tot = __shfl_sync(0xffffffffu, gi, 31);
+  *e_tot = __shfl_sync(0xffffffffu, ei, 31);
+}
+
+template <int NT, int MAXCHUNK, int SURV>
 __global__ void __cluster_dims__(kC, 1, 1) __launch_bounds__(NT, 1)
     topk_cluster_kernel(ClParams p) {
-  using SM = Smem<NT, MAXCHUNK>;
+  using SM = Smem<NT, MAXCHUNK, SURV>;
   constexpr int NW = SM::NW;
   extern __shared__ __align__(16) uint8_t smem_raw[];
   SM& S = *reinterpret_cast<SM*>(smem_raw);
@@ -139,6 +172,7 @@ __global__ void __cluster_dims__(kC, 1, 1) __launch_bounds__(NT, 1)
   const float* s = p.scores + r * p.L;
   const int lo = min(L, cta * p.chunk), hi = min(L, lo + p.chunk);
   const int w_lo = lo + warp * p.seg, w_hi = min(hi, w_lo + p.seg);   // empty when w_lo >= hi
+  const unsigned lt = (1u << lane) - 1u;
   pdl_wait();                                // the scores come from the kernel before
   pdl_release();
 
@@ -147,11 +181,11 @@ __global__ void __cluster_dims__(kC, 1, 1) __launch_bounds__(NT, 1)
     S.kmax = 0u;
     S.nsel = 0;
     S.nl = 0;
-    S.above_mine = 0;
     S.cnt_g = 0;
     S.cnt_e = 0;
   }
-  for (int i = tid; i < 2 * kBins; i += NT) (&S.hist[0][0])[i] = 0;   // both buffers
+  for (int i = tid; i < NW * kBins; i += NT) (&S.w.whist[0][0])[i] = 0;
+  for (int i = tid; i < 2 * kBins; i += NT) (&S.hist[0][0])[i] = 0;
   __syncthreads();
 
   // ---- this warp's keys; the CTA's smallest / largest selectable key
@@ -161,32 +195,53 @@ __global__ void __cluster_dims__(kC, 1, 1) __launch_bounds__(NT, 1)
     const bool vec = (reinterpret_cast<uintptr_t>(s) & 15u) == 0;   // lo, w_lo, i: multiples of 4
     const int32_t* gidx = p.gather ? p.gather + r * p.L : nullptr;
     const float* src = p.scores + r * p.src_stride;
-    for (int i = w_lo + 4 * lane; i < w_hi; i += 128) {
-      float f[4];
+    // four groups of 128 keys per step: each lane has its loads in flight
+    // before it converts any of them
+    for (int b0 = w_lo; b0 < w_hi; b0 += 4 * 128) {
+      float f[4][4];
       if (gidx) {
+        int g[4][4];
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const int g = i + u < w_hi ? __ldg(gidx + i + u) : -1;
-          f[u] = g >= 0 && g < p.src_stride ? __ldg(src + g) : __int_as_float(0xff800000);
-        }
-      } else if (vec && i + 3 < w_hi) {
-        const float4 v = __ldg(reinterpret_cast<const float4*>(s + i));
-        f[0] = v.x; f[1] = v.y; f[2] = v.z; f[3] = v.w;
+        for (int q = 0; q < 4; ++q)
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const int i = b0 + q * 128 + 4 * lane + u;
+            g[q][u] = i < w_hi ? __ldg(gidx + i) : -1;
+          }
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+#pragma unroll
+          for (int u = 0; u < 4; ++u)
+            f[q][u] = g[q][u] >= 0 && g[q][u] < p.src_stride ? __ldg(src + g[q][u]) : __int_as_float(0xff800000);
       } else {
 #pragma unroll
-        for (int u = 0; u < 4; ++u) f[u] = i + u < w_hi ? __ldg(s + i + u) : __int_as_float(0xff800000);
-      }
-      uint32_t k4[4];
+        for (int q = 0; q < 4; ++q) {
+          const int i = b0 + q * 128 + 4 * lane;
+          if (vec && i + 3 < w_hi) {
+            const float4 v = __ldg(reinterpret_cast<const float4*>(s + i));
+            f[q][0] = v.x; f[q][1] = v.y; f[q][2] = v.z; f[q][3] = v.w;
+          } else {
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        k4[u] = score_key(f[u]);
-        if (k4[u]) {
-          kmin = min(kmin, k4[u]);
-          kmax = max(kmax, k4[u]);
-          ++nsel;
+            for (int u = 0; u < 4; ++u) f[q][u] = i + u < w_hi ? __ldg(s + i + u) : __int_as_float(0xff800000);
+          }
         }
       }
-      *reinterpret_cast<uint4*>(&S.keys[i - lo]) = make_uint4(k4[0], k4[1], k4[2], k4[3]);
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const int i = b0 + q * 128 + 4 * lane;
+        if (i >= w_hi) break;                // (i - lo) stays inside the CTA's chunk
+        uint32_t k4[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          k4[u] = score_key(f[q][u]);
+          if (k4[u]) {
+            kmin = min(kmin, k4[u]);
+            kmax = max(kmax, k4[u]);
+            ++nsel;
+          }
+        }
+        *reinterpret_cast<uint4*>(&S.keys[i - lo]) = make_uint4(k4[0], k4[1], k4[2], k4[3]);
+      }
     }
     kmin = __reduce_min_sync(0xffffffffu, kmin);
     kmax = __reduce_max_sync(0xffffffffu, kmax);
@@ -221,6 +276,8 @@ __global__ void __cluster_dims__(kC, 1, 1) __launch_bounds__(NT, 1)
   uint32_t T = 0u;
   int take = 0, eqcnt = 0, cgb = 0, ceb = 0;
   bool exchange = false;                     // the counts still need an exchange
+  bool fast = false;                         // the output runs over the survivors
+  int nsurv = 0;
   if (all) {
     cgb = nsel_before;
     cluster_arrive();
@@ -237,9 +294,10 @@ __global__ void __cluster_dims__(kC, 1, 1) __launch_bounds__(NT, 1)
     int kk = p.count;
     int lowbit = 32 - common;                // key bits [lowbit-1 : 0] still undecided
     int par = 0;
-    int my_above = 0;                        // this thread's bins above the threshold bins
+    int w_above = 0, w_inbin = 0;            // this warp's keys above / in the threshold bins
     bool gathered = false;
     int ncand = 0, my_off = 0;
+    int* wh = S.w.whist[warp];
     while (lowbit > 0 && !gathered) {
       const int width = lowbit >= kDigit ? kDigit : lowbit;
       const int shift = lowbit - width;
@@ -251,59 +309,134 @@ __global__ void __cluster_dims__(kC, 1, 1) __launch_bounds__(NT, 1)
         const uint32_t kv[4] = {k4.x, k4.y, k4.z, k4.w};
 #pragma unroll
         for (int u = 0; u < 4; ++u)
-          if (kv[u] && i + u < w_hi && (kv[u] & mask) == prefix)
-            atomicAdd(&S.hist[par][(kv[u] >> shift) & dmask], 1);
+          if (kv[u] && i + u < w_hi && (kv[u] & mask) == prefix) atomicAdd(&wh[(kv[u] >> shift) & dmask], 1);
+      }
+      __syncthreads();
+      for (int b = tid; b < nb; b += NT) {   // the CTA's histogram: the warps' sum
+        int v = 0;
+#pragma unroll 8
+        for (int w = 0; w < NW; ++w) v += S.w.whist[w][b];
+        S.hist[0][b] = v;
       }
       __syncthreads();
       if (tid < kHistStores) {
         const int d = tid / (kBins / 4), q4 = 4 * (tid % (kBins / 4));
         SM* R = cl.map_shared_rank(&S, d);
-        *reinterpret_cast<int4*>(&R->inbox[par][cta][q4]) = *reinterpret_cast<const int4*>(&S.hist[par][q4]);
+        *reinterpret_cast<int4*>(&R->x.inbox[par][cta][q4]) = *reinterpret_cast<const int4*>(&S.hist[0][q4]);
       }
       cl.sync();                             // every CTA's histogram is here
       if (tid < nb) {
         int v = 0;
 #pragma unroll
-        for (int c = 0; c < kC; ++c) v += S.inbox[par][c][tid];
+        for (int c = 0; c < kC; ++c) v += S.x.inbox[par][c][tid];
         S.gsum[tid] = v;
       }
       __syncthreads();
       if (warp == 0) warp_find_bin(S.gsum, nb, kk, S);
       __syncthreads();
       const int b = S.bin;
-      if (tid < nb && tid > b) my_above += S.hist[par][tid];
       kk -= S.above;
       eqcnt = S.bin_cnt;
       prefix |= static_cast<uint32_t>(b) << shift;
       mask |= dmask << shift;
       lowbit = shift;
-      __syncthreads();                       // every thread has read the histogram
-      if (tid < kBins) S.hist[par][tid] = 0;   // zero again before its next use, two passes on
       par ^= 1;
-      if (lowbit > 0 && eqcnt <= kMaxCand) {
-        // this CTA's keys in the bin, with how many of its keys lie above it
-        for (int b0 = w_lo; b0 < w_hi; b0 += 128) {
-          const int i = b0 + 4 * lane;
-          const uint4 k4 = keys4(S, i, lo, w_hi);
-          const uint32_t kv[4] = {k4.x, k4.y, k4.z, k4.w};
-#pragma unroll
-          for (int u = 0; u < 4; ++u) {
-            const bool m = kv[u] && i + u < w_hi && (kv[u] & mask) == prefix;
-            const unsigned bal = __ballot_sync(0xffffffffu, m);
-            int base = 0;
-            if (lane == 0 && bal) base = atomicAdd(&S.nl, __popc(bal));
-            base = __shfl_sync(0xffffffffu, base, 0);
-            if (m) S.lcand[base + __popc(bal & ((1u << lane) - 1u))] = kv[u];
-          }
+      {                                      // this warp's keys above / in the bin; its histogram back to zero
+        int wa = 0, wb = 0;
+        for (int d = lane; d < nb; d += 32) {
+          const int v = wh[d];
+          wa += d > b ? v : 0;
+          wb += d == b ? v : 0;
+          wh[d] = 0;
         }
-        const int a = __reduce_add_sync(0xffffffffu, my_above);
-        if (lane == 0 && a) atomicAdd(&S.above_mine, a);
+        w_above += __reduce_add_sync(0xffffffffu, wa);
+        w_inbin = __reduce_add_sync(0xffffffffu, wb);
+      }
+      if (lowbit > 0 && eqcnt <= kMaxCand) {
+        // survivors: this CTA's keys in the bin or above it (key >= prefix)
+        if (lane == 0) {
+          S.wg[warp] = w_above + w_inbin;
+          S.we[warp] = w_above;
+        }
+        __syncthreads();                     // every warp is done with its histogram
+        int base = 0, tot = 0, above_cta = 0;
+#pragma unroll
+        for (int w = 0; w < NW; ++w) {
+          base += w < warp ? S.wg[w] : 0;
+          tot += S.wg[w];
+          above_cta += S.we[w];
+        }
+        nsurv = tot;
+        fast = tot <= SURV;                  // the same in every thread of the CTA
+        if (fast) {
+          // the survivors in position order, then the bin's keys among them
+          if (w_above + w_inbin) {
+            for (int b0 = w_lo; b0 < w_hi; b0 += 128) {
+              const int i = b0 + 4 * lane;
+              const uint4 k4 = keys4(S, i, lo, w_hi);
+              const uint32_t kv[4] = {k4.x, k4.y, k4.z, k4.w};
+              int m4 = 0;
+#pragma unroll
+              for (int u = 0; u < 4; ++u) m4 |= (kv[u] && i + u < w_hi && kv[u] >= prefix) << u;
+              // position order is lane-major: lower lanes' keys, then this
+              // lane's earlier keys, come first
+              int lower = 0, total = 0;
+#pragma unroll
+              for (int u = 0; u < 4; ++u) {
+                const unsigned bal = __ballot_sync(0xffffffffu, (m4 >> u) & 1);
+                lower += __popc(bal & lt);
+                total += __popc(bal);
+              }
+              int j = base + lower;
+#pragma unroll
+              for (int u = 0; u < 4; ++u)
+                if ((m4 >> u) & 1) {
+                  S.w.surv.key[j] = kv[u];
+                  S.w.surv.pos[j] = static_cast<uint16_t>(i + u - lo);
+                  ++j;
+                }
+              base += total;
+            }
+          }
+          __syncthreads();
+          for (int j0 = warp * 32; j0 < tot; j0 += NT) {
+            const int j = j0 + lane;
+            const uint32_t key = j < tot ? S.w.surv.key[j] : 0u;
+            const bool m = j < tot && (key & mask) == prefix;
+            const unsigned bal = __ballot_sync(0xffffffffu, m);
+            int at = 0;
+            if (lane == 0 && bal) at = atomicAdd(&S.nl, __popc(bal));
+            at = __shfl_sync(0xffffffffu, at, 0);
+            if (m) S.lcand[at + __popc(bal & lt)] = key;
+          }
+        } else {
+          // too many for the survivor buffer: the bin's keys from the whole chunk
+          int wbase = 0;
+#pragma unroll
+          for (int w = 0; w < NW; ++w) wbase += w < warp ? S.wg[w] - S.we[w] : 0;
+          if (w_inbin) {
+            for (int b0 = w_lo; b0 < w_hi; b0 += 128) {
+              const int i = b0 + 4 * lane;
+              const uint4 k4 = keys4(S, i, lo, w_hi);
+              const uint32_t kv[4] = {k4.x, k4.y, k4.z, k4.w};
+#pragma unroll
+              for (int u = 0; u < 4; ++u) {
+                const bool m = kv[u] && i + u < w_hi && (kv[u] & mask) == prefix;
+                const unsigned bal = __ballot_sync(0xffffffffu, m);
+                if (m) S.lcand[wbase + __popc(bal & lt)] = kv[u];
+                wbase += __popc(bal);
+              }
+            }
+          }
+          if (tid == 0) S.nl = tot - above_cta;
+        }
         __syncthreads();
         if (tid < kC) {
           SM* R = cl.map_shared_rank(&S, tid);
           R->x_nl[cta] = S.nl;
-          R->x_above[cta] = S.above_mine;
+          R->x_above[cta] = above_cta;
         }
+        for (int i = tid; i < 2 * kBins; i += NT) (&S.hist[0][0])[i] = 0;   // for the local passes
         cl.sync();                           // every CTA's list and count is here
         int off[kC];
         int acc = 0;
@@ -316,14 +449,14 @@ __global__ void __cluster_dims__(kC, 1, 1) __launch_bounds__(NT, 1)
         }
         ncand = acc;                         // == eqcnt
         for (int j = tid; j < ncand; j += NT) {
-          int c = 0, base = 0;               // the last CTA whose list starts at or before j
+          int c = 0, cbase = 0;              // the last CTA whose list starts at or before j
 #pragma unroll
           for (int u = 1; u < kC; ++u)
             if (j >= off[u]) {
               c = u;
-              base = off[u];
+              cbase = off[u];
             }
-          S.cand[j] = cl.map_shared_rank(S.lcand, c)[j - base];
+          S.x.cand[j] = cl.map_shared_rank(S.lcand, c)[j - cbase];
         }
         gathered = true;
         __syncthreads();
@@ -338,7 +471,7 @@ __global__ void __cluster_dims__(kC, 1, 1) __launch_bounds__(NT, 1)
         const int shift = lowbit - width;
         const uint32_t dmask = (1u << width) - 1u;
         for (int j = tid; j < ncand; j += NT) {
-          const uint32_t key = S.cand[j];
+          const uint32_t key = S.x.cand[j];
           if ((key & mask) == prefix) atomicAdd(&S.hist[lp][(key >> shift) & dmask], 1);
         }
         __syncthreads();
@@ -359,7 +492,7 @@ __global__ void __cluster_dims__(kC, 1, 1) __launch_bounds__(NT, 1)
       // candidates above / equal to T listed before this CTA's own
       int g = 0, e = 0;
       for (int j = tid; j < my_off; j += NT) {
-        const uint32_t key = S.cand[j];
+        const uint32_t key = S.x.cand[j];
         g += key > T;
         e += key == T;
       }
@@ -380,146 +513,175 @@ __global__ void __cluster_dims__(kC, 1, 1) __launch_bounds__(NT, 1)
     }
   }
 
-  // ---- per warp: keys above / equal to T.  All keys equal to T taken (the
-  // usual case): one sweep compacts each warp's picks, in order, into its own
-  // part of the key buffer (never past the keys it has read).
+  int32_t* o = p.out + r * static_cast<int64_t>(p.count);
   const bool simple = all || take >= eqcnt;
-  const uint32_t thr = all ? 1u : T;
-  const unsigned lt = (1u << lane) - 1u;
-  {
+  if (fast) {
+    // ---- ordered write over the survivors: warp w takes a run of them
+    const int per = (nsurv + NW * 32 - 1) / (NW * 32) * 32;
+    const int j_lo = min(nsurv, warp * per), j_hi = min(nsurv, j_lo + per);
     int g = 0, e = 0;
-    if (simple) {
-      for (int b0 = w_lo; b0 < w_hi; b0 += 128) {
-        const int i = b0 + 4 * lane;
-        const uint4 k4 = keys4(S, i, lo, w_hi);
-        const uint32_t kv[4] = {k4.x, k4.y, k4.z, k4.w};
-        int sel_m = 0;
-#pragma unroll
-        for (int u = 0; u < 4; ++u) sel_m |= (kv[u] >= thr && i + u < w_hi) << u;
-        if (!__any_sync(0xffffffffu, sel_m)) continue;
-        int lower = 0, total = 0;
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const unsigned sb = __ballot_sync(0xffffffffu, (sel_m >> u) & 1);
-          lower += __popc(sb & lt);
-          total += __popc(sb);
-        }
-        int q = g + lower;
-#pragma unroll
-        for (int u = 0; u < 4; ++u)
-          if ((sel_m >> u) & 1) S.keys[w_lo - lo + q++] = static_cast<uint32_t>(i + u);
-        g += total;
-      }
-    } else {
-      for (int b0 = w_lo; b0 < w_hi; b0 += 128) {
-        const int i = b0 + 4 * lane;
-        const uint4 k4 = keys4(S, i, lo, w_hi);
-        const uint32_t kv[4] = {k4.x, k4.y, k4.z, k4.w};
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const bool valid = kv[u] != 0u && i + u < w_hi;
-          g += (valid && kv[u] > T) ? 1 : 0;
-          e += (valid && kv[u] == T) ? 1 : 0;
-        }
-      }
-      g = __reduce_add_sync(0xffffffffu, g);
-      e = __reduce_add_sync(0xffffffffu, e);
+    for (int j0 = j_lo; j0 < j_hi; j0 += 32) {
+      const int j = j0 + lane;
+      const uint32_t key = j < j_hi ? S.w.surv.key[j] : 0u;
+      g += key > T ? 1 : 0;
+      e += key == T ? 1 : 0;
     }
+    g = __reduce_add_sync(0xffffffffu, g);
+    e = __reduce_add_sync(0xffffffffu, e);
     if (lane == 0) {
       S.wg[warp] = g;
       S.we[warp] = e;
     }
-  }
-  __syncthreads();
-  if (warp == 0) {
-    const int g = lane < NW ? S.wg[lane] : 0, e = lane < NW ? S.we[lane] : 0;
-    int gi = g, ei = e;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int yg = __shfl_up_sync(0xffffffffu, gi, o), ye = __shfl_up_sync(0xffffffffu, ei, o);
-      if (lane >= o) {
-        gi += yg;
-        ei += ye;
-      }
-    }
-    if (lane < NW) {
-      S.wg_off[lane] = gi - g;
-      S.we_off[lane] = ei - e;
-    }
-    const int gt = __shfl_sync(0xffffffffu, gi, 31), et = __shfl_sync(0xffffffffu, ei, 31);
-    if (exchange && lane < kC) {             // this CTA's totals to every CTA
-      SM* R = cl.map_shared_rank(&S, lane);
-      R->x_g[cta] = gt;
-      R->x_e[cta] = et;
-    }
-  }
-  if (exchange) {
-    cl.sync();                               // every CTA's counts are here
-#pragma unroll
-    for (int c = 0; c < kC; ++c) {
-      cgb += c < cta ? S.x_g[c] : 0;
-      ceb += c < cta ? S.x_e[c] : 0;
-    }
-    cluster_arrive();
-  } else {
     __syncthreads();
-  }
-
-  int32_t* o = p.out + r * static_cast<int64_t>(p.count);
-  const int g_before = cgb + S.wg_off[warp];
-  const int e_before = ceb + S.we_off[warp];
-  if (simple) {
-    const int sel_start = g_before + min(e_before, take);
-    for (int j = lane; j < S.wg[warp]; j += 32) {
-      const int q = sel_start + j;
-      const int posn = static_cast<int>(S.keys[w_lo - lo + j]);
-      if (q < p.count) o[q] = p.ids ? p.ids[r * p.L + posn] : posn;
+    if (warp == 0) {
+      int gt, et;
+      warp_offsets<SM, NW>(S, &gt, &et);
+    }
+    __syncthreads();
+    int run_eq = ceb + S.we_off[warp];
+    int run_sel = cgb + S.wg_off[warp] + min(run_eq, take);
+    for (int j0 = j_lo; j0 < j_hi; j0 += 32) {
+      const int j = j0 + lane;
+      const uint32_t key = j < j_hi ? S.w.surv.key[j] : 0u;
+      const bool eq = key == T && j < j_hi;
+      const unsigned eb = __ballot_sync(0xffffffffu, eq);
+      bool sel = key > T;
+      if (eq) sel = run_eq + __popc(eb & lt) < take;
+      const unsigned sb = __ballot_sync(0xffffffffu, sel);
+      if (sel) {
+        const int q = run_sel + __popc(sb & lt);
+        const int posn = lo + S.w.surv.pos[j];
+        if (q < p.count) o[q] = p.ids ? p.ids[r * p.L + posn] : posn;
+      }
+      run_sel += __popc(sb);
+      run_eq += __popc(eb);
     }
   } else {
-    int run_sel = g_before + min(e_before, take), run_eq = e_before;
-    for (int b0 = w_lo; b0 < w_hi; b0 += 128) {
-      const int i = b0 + 4 * lane;
-      const uint4 k4 = keys4(S, i, lo, w_hi);
-      const uint32_t kv[4] = {k4.x, k4.y, k4.z, k4.w};
-      int sel_m = 0, eq_m = 0;
+    // ---- per warp: keys above / equal to T over the whole chunk.  All keys
+    // equal to T taken (the usual case): one sweep compacts each warp's
+    // picks, in order, into its own part of the key buffer (never past the
+    // keys it has read).
+    const uint32_t thr = all ? 1u : T;
+    {
+      int g = 0, e = 0;
+      if (simple) {
+        for (int b0 = w_lo; b0 < w_hi; b0 += 128) {
+          const int i = b0 + 4 * lane;
+          const uint4 k4 = keys4(S, i, lo, w_hi);
+          const uint32_t kv[4] = {k4.x, k4.y, k4.z, k4.w};
+          int sel_m = 0;
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const bool valid = kv[u] != 0u && i + u < w_hi;
-        sel_m |= (valid && kv[u] > T) << u;
-        eq_m |= (valid && kv[u] == T) << u;
-      }
-      // position order is lane-major: lower lanes' keys, then this lane's
-      // earlier keys, come first
-      int eq_lower = 0, warp_eq = 0;
+          for (int u = 0; u < 4; ++u) sel_m |= (kv[u] >= thr && i + u < w_hi) << u;
+          if (!__any_sync(0xffffffffu, sel_m)) continue;
+          int lower = 0, total = 0;
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const unsigned eb = __ballot_sync(0xffffffffu, (eq_m >> u) & 1);
-        eq_lower += __popc(eb & lt);
-        warp_eq += __popc(eb);
-      }
-      int rank = run_eq + eq_lower;
+          for (int u = 0; u < 4; ++u) {
+            const unsigned sb = __ballot_sync(0xffffffffu, (sel_m >> u) & 1);
+            lower += __popc(sb & lt);
+            total += __popc(sb);
+          }
+          int q = g + lower;
 #pragma unroll
-      for (int u = 0; u < 4; ++u)
-        if ((eq_m >> u) & 1) {
-          if (rank < take) sel_m |= 1 << u;
-          ++rank;
+          for (int u = 0; u < 4; ++u)
+            if ((sel_m >> u) & 1) S.keys[w_lo - lo + q++] = static_cast<uint32_t>(i + u);
+          g += total;
         }
-      int sel_lower = 0, warp_sel = 0;
+      } else {
+        for (int b0 = w_lo; b0 < w_hi; b0 += 128) {
+          const int i = b0 + 4 * lane;
+          const uint4 k4 = keys4(S, i, lo, w_hi);
+          const uint32_t kv[4] = {k4.x, k4.y, k4.z, k4.w};
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const unsigned sb = __ballot_sync(0xffffffffu, (sel_m >> u) & 1);
-        sel_lower += __popc(sb & lt);
-        warp_sel += __popc(sb);
-      }
-      int pos = run_sel + sel_lower;
-#pragma unroll
-      for (int u = 0; u < 4; ++u)
-        if ((sel_m >> u) & 1) {
-          if (pos < p.count) o[pos] = p.ids ? p.ids[r * p.L + i + u] : i + u;
-          ++pos;
+          for (int u = 0; u < 4; ++u) {
+            const bool valid = kv[u] != 0u && i + u < w_hi;
+            g += (valid && kv[u] > T) ? 1 : 0;
+            e += (valid && kv[u] == T) ? 1 : 0;
+          }
         }
-      run_sel += warp_sel;
-      run_eq += warp_eq;
+        g = __reduce_add_sync(0xffffffffu, g);
+        e = __reduce_add_sync(0xffffffffu, e);
+      }
+      if (lane == 0) {
+        S.wg[warp] = g;
+        S.we[warp] = e;
+      }
+    }
+    __syncthreads();
+    if (warp == 0) {
+      int gt, et;
+      warp_offsets<SM, NW>(S, &gt, &et);
+      if (exchange && lane < kC) {           // this CTA's totals to every CTA
+        SM* R = cl.map_shared_rank(&S, lane);
+        R->x_g[cta] = gt;
+        R->x_e[cta] = et;
+      }
+    }
+    if (exchange) {
+      cl.sync();                             // every CTA's counts are here
+#pragma unroll
+      for (int c = 0; c < kC; ++c) {
+        cgb += c < cta ? S.x_g[c] : 0;
+        ceb += c < cta ? S.x_e[c] : 0;
+      }
+      cluster_arrive();
+    } else {
+      __syncthreads();
+    }
+    const int g_before = cgb + S.wg_off[warp];
+    const int e_before = ceb + S.we_off[warp];
+    if (simple) {
+      const int sel_start = g_before + min(e_before, take);
+      for (int j = lane; j < S.wg[warp]; j += 32) {
+        const int q = sel_start + j;
+        const int posn = static_cast<int>(S.keys[w_lo - lo + j]);
+        if (q < p.count) o[q] = p.ids ? p.ids[r * p.L + posn] : posn;
+      }
+    } else {
+      int run_sel = g_before + min(e_before, take), run_eq = e_before;
+      for (int b0 = w_lo; b0 < w_hi; b0 += 128) {
+        const int i = b0 + 4 * lane;
+        const uint4 k4 = keys4(S, i, lo, w_hi);
+        const uint32_t kv[4] = {k4.x, k4.y, k4.z, k4.w};
+        int sel_m = 0, eq_m = 0;
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const bool valid = kv[u] != 0u && i + u < w_hi;
+          sel_m |= (valid && kv[u] > T) << u;
+          eq_m |= (valid && kv[u] == T) << u;
+        }
+        // position order is lane-major: lower lanes' keys, then this lane's
+        // earlier keys, come first
+        int eq_lower = 0, warp_eq = 0;
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const unsigned eb = __ballot_sync(0xffffffffu, (eq_m >> u) & 1);
+          eq_lower += __popc(eb & lt);
+          warp_eq += __popc(eb);
+        }
+        int rank = run_eq + eq_lower;
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+          if ((eq_m >> u) & 1) {
+            if (rank < take) sel_m |= 1 << u;
+            ++rank;
+          }
+        int sel_lower = 0, warp_sel = 0;
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const unsigned sb = __ballot_sync(0xffffffffu, (sel_m >> u) & 1);
+          sel_lower += __popc(sb & lt);
+          warp_sel += __popc(sb);
+        }
+        int pos = run_sel + sel_lower;
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+          if ((sel_m >> u) & 1) {
+            if (pos < p.count) o[pos] = p.ids ? p.ids[r * p.L + i + u] : i + u;
+            ++pos;
+          }
+        run_sel += warp_sel;
+        run_eq += warp_eq;
+      }
     }
   }
   // padding: positions beyond the selectable keys
@@ -529,22 +691,22 @@ __global__ void __cluster_dims__(kC, 1, 1) __launch_bounds__(NT, 1)
   cluster_wait();
 }
 
-constexpr int kSmallThreads = 512, kSmallChunk = 4096;
-constexpr int kLargeThreads = 1024, kLargeChunk = 32768;
+constexpr int kSmallThreads = 512, kSmallChunk = 4096, kSmallSurv = 2048;
+constexpr int kLargeThreads = 1024, kLargeChunk = 32768, kLargeSurv = 4096;
 static_assert(kHistStores <= kSmallThreads, "one 16-byte histogram store per thread");
 
-template <int NT, int MAXCHUNK>
+template <int NT, int MAXCHUNK, int SURV>
 csa2_status launch_variant(ClParams p, int64_t rows, cudaStream_t stream) {
   constexpr int NW = NT / 32;
   const int64_t per = (p.L + kC - 1) / kC;
   p.chunk = static_cast<int>((per + 4 * NW - 1) / (4 * NW) * (4 * NW));
   p.seg = p.chunk / NW;
   if (p.chunk > MAXCHUNK) return CSA2_ERR_UNSUPPORTED;
-  using SM = Smem<NT, MAXCHUNK>;
+  using SM = Smem<NT, MAXCHUNK, SURV>;
   static std::once_flag once;
   static cudaError_t attr = cudaSuccess;
   std::call_once(once, [] {
-    attr = cudaFuncSetAttribute(topk_cluster_kernel<NT, MAXCHUNK>,
+    attr = cudaFuncSetAttribute(topk_cluster_kernel<NT, MAXCHUNK, SURV>,
                                 cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(sizeof(SM)));
   });
   if (attr != cudaSuccess) return fail(CSA2_ERR_CUDA, "select_topk_cluster: shared-memory opt-in failed");
@@ -557,7 +719,7 @@ csa2_status launch_variant(ClParams p, int64_t rows, cudaStream_t stream) {
   cfg.attrs = at;
   cfg.numAttrs = 1;
   begin_launch(stream);
-  const cudaError_t e = cudaLaunchKernelEx(&cfg, topk_cluster_kernel<NT, MAXCHUNK>, p);
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, topk_cluster_kernel<NT, MAXCHUNK, SURV>, p);
   note_launch(LK_TOPK, 1, stream);
   if (e != cudaSuccess) {
     cudaGetLastError();
@@ -586,8 +748,8 @@ csa2_status launch_select_topk_cluster(const float* scores, int64_t rows, int64_
   p.gather = gather;
   p.src_stride = gather ? src_stride : L;
   if (L <= static_cast<int64_t>(kC) * kSmallChunk)
-    return launch_variant<kSmallThreads, kSmallChunk>(p, rows, stream);
-  return launch_variant<kLargeThreads, kLargeChunk>(p, rows, stream);
+    return launch_variant<kSmallThreads, kSmallChunk, kSmallSurv>(p, rows, stream);
+  return launch_variant<kLargeThreads, kLargeChunk, kLargeSurv>(p, rows, stream);
 }
 
 }  // namespace csa2
