@@ -42,6 +42,8 @@ namespace cg = cooperative_groups;
 constexpr int kC = 8;                      // CTAs per row (one cluster)
 constexpr int kDigit = 8;
 constexpr int kBins = 1 << kDigit;         // one warp finds the bin: 8 bins per lane
+constexpr int kLocalDigit = 9;             // passes over the gathered candidates
+constexpr int kLocalBins = 1 << kLocalDigit;   // 16 bins per lane
 constexpr int kMaxCand = 4096;
 constexpr int kHistStores = kC * (kBins / 4);   // 16-byte histogram stores per CTA and pass
 
@@ -75,7 +77,7 @@ struct Smem {
       uint16_t pos[SURV];                  // their positions in the chunk
     } surv;
   } w;
-  int hist[2][kBins];                      // the CTA's histogram; the local passes' (parity)
+  int hist[2][kLocalBins];                 // the CTA's histogram; the local passes' (parity)
   int gsum[kBins];                         // the cluster's histogram
   uint32_t x_min[kC], x_max[kC];           // stored by each CTA: its selectable keys
   int x_n[kC];
@@ -95,15 +97,18 @@ __device__ __forceinline__ uint32_t score_key(float f) {
   return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
-// Warp 0 only: the bin of h[0..nb) (nb <= kBins) holding the kk-th largest
+// Warp 0 only: the bin of h[0..nb) (nb <= 32 * PER) holding the kk-th largest
 // key; sets S.bin, S.above (keys in higher bins) and S.bin_cnt.
-template <class SM>
+template <int PER, class SM>
 __device__ __forceinline__ void warp_find_bin(const int* h, int nb, int kk, SM& S) {
   const int lane = threadIdx.x & 31;
-  int v[8];
+  int v[PER];
+  int mine = 0;
 #pragma unroll
-  for (int u = 0; u < 8; ++u) v[u] = 8 * lane + u < nb ? h[8 * lane + u] : 0;
-  const int mine = v[0] + v[1] + v[2] + v[3] + v[4] + v[5] + v[6] + v[7];
+  for (int u = 0; u < PER; ++u) {
+    v[u] = PER * lane + u < nb ? h[PER * lane + u] : 0;
+    mine += v[u];
+  }
   int x = mine;                              // inclusive suffix sum over the lanes
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
@@ -112,9 +117,9 @@ __device__ __forceinline__ void warp_find_bin(const int* h, int nb, int kk, SM& 
   }
   int above = x - mine;
 #pragma unroll
-  for (int u = 7; u >= 0; --u) {
+  for (int u = PER - 1; u >= 0; --u) {
     if (above < kk && above + v[u] >= kk) {
-      S.bin = 8 * lane + u;
+      S.bin = PER * lane + u;
       S.above = above;
       S.bin_cnt = v[u];
     }
@@ -185,7 +190,7 @@ __global__ void __cluster_dims__(kC, 1, 1) __launch_bounds__(NT, 1)
     S.cnt_e = 0;
   }
   for (int i = tid; i < NW * kBins; i += NT) (&S.w.whist[0][0])[i] = 0;
-  for (int i = tid; i < 2 * kBins; i += NT) (&S.hist[0][0])[i] = 0;
+  for (int i = tid; i < 2 * kLocalBins; i += NT) (&S.hist[0][0])[i] = 0;
   __syncthreads();
 
   // ---- this warp's keys; the CTA's smallest / largest selectable key
@@ -332,7 +337,7 @@ __global__ void __cluster_dims__(kC, 1, 1) __launch_bounds__(NT, 1)
         S.gsum[tid] = v;
       }
       __syncthreads();
-      if (warp == 0) warp_find_bin(S.gsum, nb, kk, S);
+      if (warp == 0) warp_find_bin<kBins / 32>(S.gsum, nb, kk, S);
       __syncthreads();
       const int b = S.bin;
       kk -= S.above;
@@ -359,12 +364,22 @@ __global__ void __cluster_dims__(kC, 1, 1) __launch_bounds__(NT, 1)
           S.we[warp] = w_above;
         }
         __syncthreads();                     // every warp is done with its histogram
-        int base = 0, tot = 0, above_cta = 0;
+        int base, tot, above_cta, cand_before;
+        {                                    // every warp: scan over the warps' counts
+          const int sv = lane < NW ? S.wg[lane] : 0, av = lane < NW ? S.we[lane] : 0;
+          int si = sv, ci = sv - av;
 #pragma unroll
-        for (int w = 0; w < NW; ++w) {
-          base += w < warp ? S.wg[w] : 0;
-          tot += S.wg[w];
-          above_cta += S.we[w];
+          for (int o = 1; o < 32; o <<= 1) {
+            const int ys = __shfl_up_sync(0xffffffffu, si, o), yc = __shfl_up_sync(0xffffffffu, ci, o);
+            if (lane >= o) {
+              si += ys;
+              ci += yc;
+            }
+          }
+          base = __shfl_sync(0xffffffffu, si - sv, warp);
+          cand_before = __shfl_sync(0xffffffffu, ci - (sv - av), warp);
+          tot = __shfl_sync(0xffffffffu, si, 31);
+          above_cta = __reduce_add_sync(0xffffffffu, av);
         }
         nsurv = tot;
         fast = tot <= SURV;                  // the same in every thread of the CTA
@@ -411,9 +426,7 @@ __global__ void __cluster_dims__(kC, 1, 1) __launch_bounds__(NT, 1)
           }
         } else {
           // too many for the survivor buffer: the bin's keys from the whole chunk
-          int wbase = 0;
-#pragma unroll
-          for (int w = 0; w < NW; ++w) wbase += w < warp ? S.wg[w] - S.we[w] : 0;
+          int wbase = cand_before;
           if (w_inbin) {
             for (int b0 = w_lo; b0 < w_hi; b0 += 128) {
               const int i = b0 + 4 * lane;
@@ -436,7 +449,7 @@ __global__ void __cluster_dims__(kC, 1, 1) __launch_bounds__(NT, 1)
           R->x_nl[cta] = S.nl;
           R->x_above[cta] = above_cta;
         }
-        for (int i = tid; i < 2 * kBins; i += NT) (&S.hist[0][0])[i] = 0;   // for the local passes
+        for (int i = tid; i < 2 * kLocalBins; i += NT) (&S.hist[0][0])[i] = 0;   // for the local passes
         cl.sync();                           // every CTA's list and count is here
         int off[kC];
         int acc = 0;
@@ -467,7 +480,7 @@ __global__ void __cluster_dims__(kC, 1, 1) __launch_bounds__(NT, 1)
       // further passes over the candidates alone (both histograms are zero)
       int lp = 0;
       while (lowbit > 0) {
-        const int width = lowbit >= kDigit ? kDigit : lowbit;
+        const int width = lowbit >= kLocalDigit ? kLocalDigit : lowbit;
         const int shift = lowbit - width;
         const uint32_t dmask = (1u << width) - 1u;
         for (int j = tid; j < ncand; j += NT) {
@@ -475,7 +488,7 @@ __global__ void __cluster_dims__(kC, 1, 1) __launch_bounds__(NT, 1)
           if ((key & mask) == prefix) atomicAdd(&S.hist[lp][(key >> shift) & dmask], 1);
         }
         __syncthreads();
-        if (warp == 0) warp_find_bin(S.hist[lp], 1 << width, kk, S);
+        if (warp == 0) warp_find_bin<kLocalBins / 32>(S.hist[lp], 1 << width, kk, S);
         __syncthreads();
         prefix |= static_cast<uint32_t>(S.bin) << shift;
         mask |= dmask << shift;
@@ -484,7 +497,7 @@ __global__ void __cluster_dims__(kC, 1, 1) __launch_bounds__(NT, 1)
         lowbit = shift;
         // zero for the pass after next, whose counts start after the next
         // pass's first barrier
-        if (tid < kBins) S.hist[lp][tid] = 0;
+        for (int i = tid; i < kLocalBins; i += NT) S.hist[lp][i] = 0;
         lp ^= 1;
       }
       T = prefix;
