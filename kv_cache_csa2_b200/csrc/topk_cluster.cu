@@ -16,15 +16,20 @@
 // round trip; a store does not wait):
 //   1. each CTA's smallest / largest selectable key and count go to every CTA;
 //   2. radix passes of 8-bit digits below the bits all selectable keys share:
-//      each CTA histograms its keys and stores the histogram into every CTA,
-//      so every CTA sums the same eight histograms and takes the same bin;
-//   3. once the threshold bin holds at most kMaxCand keys, each CTA lists its
-//      keys in that bin and every CTA copies the eight lists (in CTA order);
-//      the remaining 8-bit passes run over the candidates alone;
+//      each warp counts its keys into its own histogram, the CTA's sum is
+//      stored into every CTA, so every CTA sums the same eight histograms and
+//      takes the same bin;
+//   3. once the threshold bin holds at most kMaxCand keys, each CTA compacts
+//      its keys in or above the bin (the survivors, in position order, with
+//      their positions; the per-warp histograms give each warp its offset),
+//      lists the bin's keys, and every CTA copies the eight lists (in CTA
+//      order); the remaining passes (9-bit digits) run over the candidates;
 //   4. each CTA's output offset follows from the counts it has: the keys above
 //      the threshold bins in the CTAs before it (sent with the lists) and the
-//      candidates before its own in the copied list.  Only a row whose
-//      threshold bin never fits the list needs one more exchange of counts.
+//      candidates before its own in the copied list; the ordered write runs
+//      over the survivors.  A CTA with more survivors than its buffer holds
+//      sweeps its whole chunk instead, and only a row whose threshold bin
+//      never fits the list needs one more exchange of counts.
 // Integer counts only: the result is deterministic.
 #include <cooperative_groups.h>
 
