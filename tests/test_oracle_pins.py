@@ -205,6 +205,27 @@ def test_pool_contains_topk():
         assert set(top[r]) <= set(pool[r])
 
 
+def test_topk_of_pool_is_topk_of_row():
+    """The reading a Full layer's two-step selection rests on: selecting the
+    k best inside the P best (k <= P), through the pool's positions, gives
+    exactly the row's k best (same order and ties, -inf never chosen, pools
+    padded with -1 when fewer than P entries are selectable)."""
+    rng = np.random.default_rng(7)
+    for trial in range(200):
+        L = int(rng.integers(1, 400))
+        s = rng.integers(-4, 4, size=(2, L)).astype(float)     # heavy ties
+        s[rng.random((2, L)) < 0.3] = -np.inf
+        if trial % 3 == 0:
+            s = rng.standard_normal((2, L)).round(1)
+        P = int(rng.integers(1, L + 50))
+        k = int(rng.integers(1, P + 1))
+        pool = O.select_top(s, P)
+        g = np.where(pool >= 0, np.take_along_axis(s, np.maximum(pool, 0), 1), -np.inf)
+        pos = O.select_top(g, k)
+        two_step = np.where(pos >= 0, np.take_along_axis(pool, np.maximum(pos, 0), 1), -1)
+        assert np.array_equal(two_step, O.select_top(s, k)), (trial, L, P, k)
+
+
 # ----------------------------------------------------------------------------- attention
 
 def test_attn_golden():
