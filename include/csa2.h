@@ -132,7 +132,9 @@ csa2_status csa2_index_scores(const void* q, const float* w, const void* k, int 
  * are selected together.
  *
  *   scores f32 [rows, L]    ids int32 [rows, L] or NULL    out int32 [rows, count]
- *   workspace: csa2_select_topk_workspace(rows, L, count) bytes of device memory.
+ *   workspace: csa2_select_topk_workspace(rows, L, count) bytes of device memory
+ *   (an upper bound: with fewer rows than the GPU has SMs and L <= 262144 the
+ *   selection runs on clusters of CTAs and uses none of it).
  */
 size_t csa2_select_topk_workspace(int64_t rows, int64_t L, int count);
 csa2_status csa2_select_topk(const float* scores, int64_t rows, int64_t L, int count,
