@@ -17,8 +17,9 @@ timed region ("e2e"), the dominant kernel's roofline from live per-kernel
 event timing, the SM clocks sampled during the timed region, and the CPU
 oracle on a bounded sample ("cpu_baseline").
 
---impl reference times the float64 CPU oracle on the same workload, one
-query's layer group per step, on rank 0 only.
+--impl reference times the float64 CPU oracle on the same workload, the GPU
+arm's whole batch per step (a spread sample of 8 queries for the 4096-query
+prefill), on rank 0 only.
 
 Multi-GPU (torchrun): every rank runs its own replica of the workload; the
 path has no data-path collective (sequences are independent).
@@ -44,6 +45,8 @@ METRIC = "CSA2 decode queries/s per layer group at 1M ctx; achieved HBM TB/s vs 
 UNIT = "queries/s"
 L2_BYTES = 126 * 2 ** 20
 FALLBACK_HBM_GBS = 6650.0
+REF_MAX_BATCH = 64        # largest batch the reference arm runs whole per step
+REF_SAMPLE = 8            # queries per reference step of a larger batch (prefill)
 
 
 # ---------------------------------------------------------------------------- ranks
@@ -144,6 +147,17 @@ def measured_hbm_gbs():
         return FALLBACK_HBM_GBS, "fallback"
 
 
+def measured_tflops(launch_s):
+    """Dense bf16 tensor peak: the burst figure for a launch shorter than 1 ms,
+    the sustained (power-capped) one for longer launches."""
+    key = "bf16_tflops_sustained" if launch_s >= 1e-3 else "bf16_tflops"
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return float(json.load(f)[key]), f"measured (MEASURED_PEAKS.json {key})"
+    except (OSError, KeyError, ValueError):
+        return (1400.0 if launch_s >= 1e-3 else 1590.0), "fallback (pool's earlier measurement)"
+
+
 def source_digest(*names) -> str:
     h = hashlib.sha256()
     for n in names:
@@ -200,6 +214,30 @@ def algorithmic_bytes(wl):
         out["index_pool"] = (n_re * (rows * wl.P * (wl.d * 2 + 4) + qidx), n_re)
     attn = wl.n_layers * (rows * wl.k * (kv_row + 4) + rows * wl.Ha * (wl.D * 2 * 2 + 4))
     out["attn"] = (attn, wl.n_layers)
+    if wl.compress_new_tokens:        # raw tokens c (bf16) and z (f32) in, entries (bf16) out
+        t_in = wl.compress_new_tokens + (wl.m if wl.halo else 0)
+        n_new = wl.compress_new_tokens // wl.m
+        out["compress"] = (wl.B * (t_in * wl.D * 6 + n_new * wl.D * 2) + 2 * wl.m * wl.D * 4, 1)
+    return out
+
+
+def algorithmic_flops(wl):
+    """Tensor-core work the method must do in one step, per kernel kind: the
+    indexer's q.k products over the scored entries (Full: every visible entry,
+    causal in prefill; Reindex: the pool) and attention's two products over
+    the selected rows.  {kind: flops per step}."""
+    import numpy as np
+    from kv_cache_csa2_b200.configs import n_visible
+    rows = wl.B * wl.Q
+    nv = n_visible(wl)
+    visible = int(np.asarray(nv, dtype=np.int64).sum()) if nv is not None else rows * wl.N
+    n_full = sum(1 for m in wl.modes if m == "full")
+    n_re = sum(1 for m in wl.modes if m == "reindex")
+    per = 2 * wl.Hi * wl.d
+    out = {"index_scores": per * visible * (n_full + (n_re if wl.P == 0 else 0))}
+    if wl.P and n_re:
+        out["index_pool"] = per * rows * wl.P * n_re
+    out["attn"] = wl.n_layers * rows * wl.k * wl.Ha * wl.D * 4
     return out
 
 
@@ -252,6 +290,22 @@ def run_ours(args, wl, world, rank, local):
     inp = I.make_inputs(wl, seed=args.seed)
     D = device_inputs(wl, inp, torch, dev)
     kv, kv_scales = D["kv"], None
+    compress = None
+    if wl.compress_new_tokens:
+        # the newest entries are compressed from raw tokens inside every step
+        # (row a1), appended after the cached entries of the KV buffer
+        n_cached = inp["kv"].shape[1]
+        kv = torch.empty(wl.B, wl.N, wl.D, dtype=torch.bfloat16, device=dev)
+        kv[:, :n_cached] = D["kv"]
+        del D["kv"]
+        bf = lambda bits: torch.from_numpy(bits.view("int16")).view(torch.bfloat16).to(dev)  # noqa: E731
+        D["c"], D["z"] = bf(inp["c"]), torch.from_numpy(inp["z"]).to(dev)
+        D["bias"] = torch.from_numpy(inp["bias"]).to(dev)
+        tail = kv[:, n_cached:]
+
+        def compress():
+            K.csa2_compress(D["c"], D["z"], D["bias"], wl.m, has_left_halo=wl.halo, out=tail,
+                            out_batch_stride=wl.N * wl.D)
     if wl.kv_fp4:
         kv, kv_scales = K.csa2_fp4_pack(D["kv"])
     modes = [{"full": K.FULL, "reindex": K.REINDEX, "reuse": K.REUSE}[m] for m in wl.modes]
@@ -272,6 +326,8 @@ def run_ours(args, wl, world, rank, local):
         kws.append(kw)
 
     def layer(i):
+        if i == 0 and compress is not None:
+            compress()
         g.layer(i, D["layers"][i]["q_attn"], outs[i], lses[i], **kws[i])
 
     flush_buf = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device=dev)
@@ -377,6 +433,10 @@ def run_ours(args, wl, world, rank, local):
     # outputs come back on another while layer i+1 computes (a step starts
     # after the previous step's compute and copies).
     h_in, d_in = [[] for _ in range(n_layers)], [[] for _ in range(n_layers)]
+    if compress is not None:          # the step's raw tokens go up with the first layer's queries
+        for key in ("c", "z"):
+            h_in[0].append(D[key].cpu().pin_memory())
+            d_in[0].append(D[key])
     for i in range(n_layers):
         for key in ("q_attn", "q_index", "w_index"):
             t = D["layers"][i].get(key)
@@ -432,15 +492,26 @@ def run_ours(args, wl, world, rank, local):
     if dom is not None:
         tot_ms, n = per_kind[dom]
         avg_s = tot_ms / n / 1e3
-        step_bytes = kernel_min_bytes(wl).get(dom, 0)
-        bytes_per_launch = step_bytes / max(n / args.steps, 1)
-        achieved = bytes_per_launch / avg_s / 1e9 if avg_s > 0 else 0.0
-        roof = {"kernel": dom, "bound": "hbm", "achieved": round(achieved, 1), "peak": hbm,
-                "unit": "GB/s", "frac": round(achieved / hbm, 4), "traffic": ncu_traffic(dom),
-                "algorithmic_bytes_per_launch": int(bytes_per_launch),
-                "avg_launch_us": round(avg_s * 1e6, 2), "launches": n,
-                "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs)" if peak_src == "measured"
-                else "fallback 6650 GB/s"}
+        per_step = n / args.steps
+        bytes_per_launch = kernel_min_bytes(wl).get(dom, 0) / max(per_step, 1)
+        flops_per_launch = algorithmic_flops(wl).get(dom, 0) / max(per_step, 1)
+        tflops, tf_src = measured_tflops(avg_s)
+        # the bound is whichever of the two ideal times is longer
+        tensor = flops_per_launch / (tflops * 1e12) > bytes_per_launch / (hbm * 1e9)
+        if tensor:
+            achieved = flops_per_launch / avg_s / 1e12 if avg_s > 0 else 0.0
+            roof = {"kernel": dom, "bound": "tensor", "achieved": round(achieved, 1), "peak": tflops,
+                    "unit": "TFLOP/s", "frac": round(achieved / tflops, 4), "traffic": ncu_traffic(dom),
+                    "algorithmic_flops_per_launch": int(flops_per_launch),
+                    "algorithmic_bytes_per_launch": int(bytes_per_launch), "peak_source": tf_src}
+        else:
+            achieved = bytes_per_launch / avg_s / 1e9 if avg_s > 0 else 0.0
+            roof = {"kernel": dom, "bound": "hbm", "achieved": round(achieved, 1), "peak": hbm,
+                    "unit": "GB/s", "frac": round(achieved / hbm, 4), "traffic": ncu_traffic(dom),
+                    "algorithmic_bytes_per_launch": int(bytes_per_launch),
+                    "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs)" if peak_src == "measured"
+                    else "fallback 6650 GB/s"}
+        roof.update(avg_launch_us=round(avg_s * 1e6, 2), launches=n)
     kernels = {k: {"total_ms": round(v[0], 4), "launches": v[1],
                    "avg_us": round(v[0] / v[1] * 1e3, 2)} for k, v in per_kind.items()}
     total_alg = sum(v[0] for v in alg.values())
@@ -488,20 +559,22 @@ def run_ours(args, wl, world, rank, local):
 # ---------------------------------------------------------------------------- oracle (CPU)
 
 def oracle_queries(wl, inp, queries):
-    """Run the oracle's layer group for the listed (b, q) queries; returns seconds."""
+    """Run the oracle's layer group for the listed (b, q) queries (each
+    sequence's raw tokens compressed once per call); returns seconds."""
     import numpy as np
     import oracle as O
     from kv_cache_csa2_b200 import inputs as I
 
     t0 = time.perf_counter()
     n_cached = inp["kv"].shape[1]
+    new_of = {}
     for b, t in queries:
         kb = inp["kv"][b:b + 1]
-        new = None
-        if wl.compress_new_tokens:         # the newest entries come from raw tokens: compress them
-            _, new = O.compress(O.bf16_bits_to_float(inp["c"][b:b + 1]),
-                                inp["z"][b:b + 1].astype(np.float64),
-                                inp["bias"].astype(np.float64), wl.m, wl.halo)
+        if wl.compress_new_tokens and b not in new_of:   # the newest entries come from raw tokens
+            _, new_of[b] = O.compress(O.bf16_bits_to_float(inp["c"][b:b + 1]),
+                                      inp["z"][b:b + 1].astype(np.float64),
+                                      inp["bias"].astype(np.float64), wl.m, wl.halo)
+        new = new_of.get(b)
 
         def rows(_, ids, kb=kb, new=new):
             ids = np.asarray(ids)
@@ -539,7 +612,8 @@ def cpu_baseline(wl, inp, budget_s=20.0):
     while done < len(qs) and spent < budget_s:
         spent += oracle_queries(wl, inp, [qs[done]])
         done += 1
-    return {"value": round(done / spent, 3), "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+    return {"value": round(done / spent, 3), "unit": UNIT, "cores": os.cpu_count() or 1,
+            "blas_threads": blas_threads(), "kind": "oracle",
             "sample": f"{done} of the workload's {len(qs)} queries, each through the whole layer group "
                       f"(float64 numpy oracle), {spent:.1f} s"}
 
@@ -550,14 +624,24 @@ def run_reference(args, wl, world, rank):
     from kv_cache_csa2_b200 import inputs as I
     inp = I.make_inputs(wl, seed=args.seed)
     qs = [(b, t) for b in range(wl.B) for t in range(wl.Q)]
-    for i in range(args.warmup):
+    # a step is the GPU arm's whole batch when it has at most REF_MAX_BATCH
+    # queries (every decode workload), else REF_SAMPLE queries spread over it
+    if len(qs) <= REF_MAX_BATCH:
+        per_step, same = len(qs), True
+    else:
+        per_step, same = REF_SAMPLE, False
+    stride = max(1, len(qs) // per_step)
+    for i in range(args.warmup):            # warm-up: one query each (untimed)
         oracle_queries(wl, inp, [qs[i % len(qs)]])
-    spent = 0.0
+    spent, done = 0.0, 0
     for i in range(args.steps):
-        spent += oracle_queries(wl, inp, [qs[i % len(qs)]])
-    value = args.steps / spent
-    cores = blas_threads()
-    sample = f"{args.steps} single-query layer groups of the workload (float64 numpy oracle)"
+        batch = [qs[(i + j * stride) % len(qs)] for j in range(per_step)]
+        spent += oracle_queries(wl, inp, batch)
+        done += len(batch)
+    value = done / spent
+    cores = os.cpu_count() or 1
+    sample = (f"{args.steps} steps of {per_step} queries, each through the whole layer group "
+              f"(float64 numpy oracle){'' if same else f'; the workload has {len(qs)} queries per step'}")
     return {"impl": "reference", "metric": METRIC, "value": round(value, 3), "unit": UNIT,
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": round(spent / args.steps * 1e3, 3), "higher_is_better": True,
@@ -565,9 +649,9 @@ def run_reference(args, wl, world, rank):
             "data": "synthetic (seeded N(0,1)/U(0,1) inputs of the workload's shapes)",
             "config": {"workload": wl.name, "B": wl.B, "Q": wl.Q, "L": wl.L, "N": wl.N, "D": wl.D,
                        "k": wl.k, "P": wl.P, "modes": ",".join(wl.modes),
-                       "sample_per_step": "one query"},
+                       "sample_per_step": f"{per_step} queries" + (" (the whole batch)" if same else "")},
             "cpu_baseline": {"value": round(value, 3), "unit": UNIT, "cores": cores,
-                             "kind": "oracle", "sample": sample},
+                             "blas_threads": blas_threads(), "kind": "oracle", "sample": sample},
             "e2e": {"value": round(value, 3), "unit": UNIT, "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
 

@@ -147,9 +147,13 @@ csa2_status csa2_select_topk(const float* scores, int64_t rows, int64_t L, int c
  * of csa2_select_topk (same kernels, bit-identical output); the scratch is a
  * static device array of CSA2_SELECT_TOPK_NOALLOC_SCRATCH_BYTES per device
  * inside the library, so the call allocates nothing.
- *   - A selection that needs more scratch than that (csa2_select_topk_workspace
- *     of the same arguments) returns CSA2_ERR_OOM with nothing enqueued; at
- *     L = 262144 the limit is about 40 rows.
+ *   - Only the kernel with several cooperating CTAs per row uses scratch
+ *     (rows of more than 262144 keys, or at least as many rows as the GPU has
+ *     SMs with more than 32768 keys); it needs about 164 KiB per row, so at
+ *     most 25 rows fit.  A call on that path that needs more than the array
+ *     returns CSA2_ERR_OOM with nothing enqueued.  The paths that keep their
+ *     state in shared memory (fewer rows than SMs and L <= 262144; L <= 32768)
+ *     need no scratch and have no such limit.
  *   - The part of the scratch that must start at zero is cleared on `stream`
  *     before every launch (an asynchronous memset, no allocation).
  *   - The scratch is shared: calls that overlap on one device (other streams,
@@ -298,6 +302,16 @@ void csa2_reset_launch_counts(void);
 csa2_status csa2_timing_enable(int on);
 int csa2_kernel_times(double* ms, int64_t* launches, int n);
 void csa2_timing_reset(void);
+/* Bound of the device waits in which one CTA waits for another: the row
+ * barrier of the multi-CTA top-k and the attention kernel's wait for another
+ * tile's partial.  Such a wait gives up after limit_ns nanoseconds (0 = the
+ * default, one second), records CSA2_ERR_TIMEOUT in the device error word,
+ * and the kernel then finishes its remaining steps without waiting again on
+ * the CTA it gave up on, so it ends and leaves the context usable (its
+ * results are then undefined).  With unreachable != 0 those waits target a
+ * count that no CTA writes, so each one runs out: a test of the error path
+ * without a fault.  Applies to launches enqueued after the call; process-wide. */
+csa2_status csa2_set_device_wait(uint64_t limit_ns, int unreachable);
 /* Host-side fault injection for tests: "alloc", "launch" or "" (off).  While
  * set, every call returns CSA2_ERR_OOM / CSA2_ERR_CUDA before touching the
  * device.  The environment variable CSA2_FAULT sets the initial value. */

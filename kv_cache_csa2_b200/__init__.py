@@ -15,7 +15,7 @@ __all__ = [
     "ACT_IDENTITY", "csa2_compress", "csa2_index_scores", "csa2_select_topk", "csa2_select_topk_noalloc",
     "csa2_index_topk",
     "csa2_sparse_attn", "csa2_fp4_pack", "csa2_fp4_unpack", "Group", "csa2_device_error",
-    "launch_counts", "reset_launch_counts", "set_fault", "EXPORTED_SYMBOLS",
+    "launch_counts", "reset_launch_counts", "set_fault", "set_device_wait", "EXPORTED_SYMBOLS",
 ]
 
 FULL, REINDEX, REUSE = 0, 1, 2
@@ -68,6 +68,7 @@ _SIGS = {
     "csa2_launch_counts": (_I, [ctypes.POINTER(_I64), _I]),
     "csa2_reset_launch_counts": (None, []),
     "csa2_set_fault": (_I, [ctypes.c_char_p]),
+    "csa2_set_device_wait": (_I, [ctypes.c_uint64, _I]),
     "csa2_timing_enable": (_I, [_I]),
     "csa2_kernel_times": (_I, [ctypes.POINTER(ctypes.c_double), ctypes.POINTER(_I64), _I]),
     "csa2_timing_reset": (None, []),
@@ -367,3 +368,9 @@ def kernel_times() -> dict:
 
 def set_fault(kind: str) -> None:
     _check(lib().csa2_set_fault(kind.encode()))
+
+
+def set_device_wait(limit_ns: int = 0, unreachable: bool = False) -> None:
+    """Bound of the cross-CTA device waits (0 = default, 1 s); `unreachable`
+    makes each such wait run out (a test of the error path)."""
+    _check(lib().csa2_set_device_wait(int(limit_ns), int(bool(unreachable))))

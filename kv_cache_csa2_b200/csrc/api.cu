@@ -116,13 +116,22 @@ void note_launch(LaunchKind kind, int n, cudaStream_t s) {
 __device__ int g_dev_err;
 
 static std::mutex g_dev_mu;
-static int* g_err_ptr[64];
-static int g_sms[64];
+static int* g_err_ptr[kMaxDevices];
+static int g_sms[kMaxDevices];
 
 static int current_device() {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return 0;
-  return dev < 64 ? dev : 63;
+  return dev < kMaxDevices ? dev : kMaxDevices - 1;
+}
+
+int current_device_or_none() {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) {
+    cudaGetLastError();
+    return -1;
+  }
+  return dev >= 0 && dev < kMaxDevices ? dev : -1;
 }
 
 int* device_error_word() {
@@ -142,6 +151,19 @@ int* device_error_word() {
 bool pdl_enabled() {
   static const bool on = getenv("CSA2_NO_PDL") == nullptr;
   return on;
+}
+
+// ------------------------------------------------------ cross-CTA wait bound
+static std::atomic<unsigned long long> g_wait_ns{0};     // 0: the default
+static std::atomic<int> g_wait_unreachable{0};
+
+unsigned long long cross_cta_wait_ns() {
+  const unsigned long long v = g_wait_ns.load(std::memory_order_relaxed);
+  return v ? v : kDefaultCrossCtaWaitNs;
+}
+
+unsigned cross_cta_wait_offset() {
+  return g_wait_unreachable.load(std::memory_order_relaxed) ? kUnreachableWaitOffset : 0u;
 }
 
 int sm_count() {
@@ -212,6 +234,12 @@ const char* csa2_status_string(csa2_status s) {
 const char* csa2_last_error(void) { return t_msg; }
 
 int csa2_version(void) { return 1; }
+
+csa2_status csa2_set_device_wait(uint64_t limit_ns, int unreachable) {
+  g_wait_ns.store(limit_ns);
+  g_wait_unreachable.store(unreachable ? 1 : 0);
+  return CSA2_OK;
+}
 
 csa2_status csa2_set_fault(const char* kind) {
   const int f = parse_fault(kind);

@@ -29,9 +29,10 @@
 //              into the 128-byte-swizzled layout, 64 per thread in flight; the
 //              next wave's gather is issued as soon as this wave's products are
 //              done), softmax, partial write, flag waits, reduction, output.
-// Every wait is bounded (mbarriers 2 s, the flags 1 s); a CTA that gives up
-// records CSA2_ERR_TIMEOUT and still takes every later step, so no other CTA
-// waits for it in vain.
+// Every wait is bounded (mbarriers 2 s, the flags 1 s or the host-set bound);
+// a CTA that gives up records CSA2_ERR_TIMEOUT and still takes every later
+// step, so no other CTA waits for it in vain, and before it exits it waits
+// (bounded) for its own copies and products in flight.
 #include <algorithm>
 #include <cstdlib>
 #include <cstring>
@@ -86,6 +87,8 @@ struct Params {
   int Q, k, T, G, dpc;
   int bulk;                        // a CTA's dims of all T partials fit the KV region, their (m, l) the P region
   float scale;
+  unsigned long long wait_ns;      // bound of the wait for another tile's partial
+  unsigned wait_offset;            // added to the awaited count (0, or unreachable for tests)
 };
 
 // Reduce 64 per-thread values over the 32 lanes of a warp (max or sum): five
@@ -160,6 +163,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* m_done = bar + 4;                  // the reduction no longer needs the q region
   uint64_t* r_full = bar + 5;                  // this CTA's dims of every partial are in the KV region
   uint64_t* kv_full = bar + 8;                 // [8]: one per 64-column block of the tile
+  uint64_t* mma_fin = bar + 3;                 // every MMA of this CTA has completed (teardown)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + OFF_MISC + 4);
 
@@ -193,6 +197,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int mc = 0; mc < 4; ++mc) mbar_init(&o_full[mc], 1);
     mbar_init(m_done, 1);
     mbar_init(r_full, 1);
+    mbar_init(mma_fin, 1);
     for (int kb = 0; kb < kKB; ++kb) mbar_init(&kv_full[kb], 128);
     *abort_flag = 0;
     fence_mbar_init();
@@ -261,6 +266,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                      desc_mnmajor_sw128(p0 + kk * 2048, 8192, 1024), idesc_o, kk != 0);
           mma_commit(&o_full[mc]);                 // chunk mc can be read while mc+1 computes
         }
+      }
+      // before TMEM is freed, every product issued above has completed, also
+      // when a wait gave up on the way (bounded: 0.1 s)
+      mma_commit(mma_fin);
+      const uint64_t t0 = globaltimer_ns();
+      while (!mbar_try_wait(mma_fin, 0) && globaltimer_ns() - t0 < 100000000ull) {
       }
     }
     __syncwarp();
@@ -429,11 +440,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       // is resident: the launch is cooperative) and, on the bulk path, loads
       // this CTA's dims of it and its (m, l) at once
       if (et < p.T) {
-        const unsigned gen = sh_gen;
+        const unsigned gen = sh_gen + p.wait_offset;
         const unsigned* fj = p.flag + (blockIdx.x - tile) + et;
         const uint64_t t0 = globaltimer_ns();
         while (static_cast<int>(ld_acquire_u32(fj) - gen) < 0) {
-          if (globaltimer_ns() - t0 > 1000000000ull) {
+          if (globaltimer_ns() - t0 > p.wait_ns) {
             raise_dev_error(p.err, DEVERR_TIMEOUT);
             *abort_flag = 1;
             break;
@@ -449,7 +460,16 @@ __global__ void __launch_bounds__(kThreads, 1)
       epi_bar();
       // weights of the T partials exp(m_j - M), the query's M and L
       if (p.bulk) {
-        ok = mbar_wait(r_full, par, abort_flag, p.err) && ok;
+        // the copies read memory that exists whatever the flags said, so they
+        // all land: wait for them also after a give-up (bounded: 0.1 s), so
+        // that no copy is in flight when the region is reused or the CTA exits
+        {
+          const uint64_t t0 = globaltimer_ns();
+          bool landed;
+          while (!(landed = mbar_try_wait(r_full, par)) && globaltimer_ns() - t0 < 100000000ull) {
+          }
+          ok = ok && landed;
+        }
         // all 128 threads: head h = et % 64 takes tiles j = half, half + 2, ...
         // (half = et / 64); every load is issued before any is used
         {
@@ -618,9 +638,8 @@ Shape shape_for(int k) {
 // CTAs of this kernel that fit on the device at once (cached), capped by the
 // environment variable CSA2_ATTN_MAX_CTAS (tests: several waves per launch).
 int resident_ctas() {
-  static std::once_flag once;
-  static int cap = 0;
-  std::call_once(once, [] {
+  static PerDevice<int> cache;
+  int c = cache.get([] {
     int per_sm = 0;
     if (cudaFuncSetAttribute(attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES) !=
             cudaSuccess ||
@@ -629,9 +648,8 @@ int resident_ctas() {
       cudaGetLastError();
       per_sm = 0;
     }
-    cap = std::min(per_sm * sm_count(), kAttnMaxGrid);
+    return std::min(per_sm * sm_count(), kAttnMaxGrid);
   });
-  int c = cap;
   if (const char* e = getenv("CSA2_ATTN_MAX_CTAS")) {
     const int v = atoi(e);
     if (v > 0) c = std::min(c, v);
@@ -704,6 +722,8 @@ csa2_status launch_sparse_attn_tc(const void* q, const csa2_kv& kv, const int32_
   p.dpc = s.dpc;
   p.bulk = static_cast<int64_t>(s.T) * s.dpc * HA * 4 <= kKB * kKBBytes && s.T * 2 * HA * 4 <= kRows * 128;
   p.scale = scale;
+  p.wait_ns = cross_cta_wait_ns();
+  p.wait_offset = cross_cta_wait_offset();
   if (!sync_zeroed) {          // a caller workspace: flags start at zero
     begin_launch(stream);
     if (cudaMemsetAsync(p.flag, 0, static_cast<size_t>(G) * s.T * 4, stream) != cudaSuccess)

@@ -6,6 +6,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <mutex>
+
 #include "csa2.h"
 
 namespace csa2 {
@@ -39,6 +41,24 @@ csa2_status fault_gate();
 int* device_error_word();
 // Number of SMs of the current device (cached per device).
 int sm_count();
+// Ordinal of the current device, or -1 when it cannot be read or is >= kMaxDevices.
+constexpr int kMaxDevices = 64;
+int current_device_or_none();
+
+// A value computed once per device, with that device current (a kernel's
+// shared-memory opt-in or its occupancy binds to the device current when it
+// is made).  Devices past kMaxDevices recompute it on every call.
+template <class T>
+struct PerDevice {
+  std::once_flag once[kMaxDevices];
+  T value[kMaxDevices] = {};
+  T get(T (*make)()) {
+    const int dev = current_device_or_none();
+    if (dev < 0) return make();
+    std::call_once(once[dev], [this, dev, make] { value[dev] = make(); });
+    return value[dev];
+  }
+};
 
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -51,6 +71,16 @@ inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 __device__ __forceinline__ void pdl_release() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 bool pdl_enabled();
+
+// Bound of the waits in which one CTA waits for another (the multi-CTA top-k
+// row barrier, the attention kernel's wait for another tile's partial):
+// csa2_set_device_wait() sets it, by default one second.  A kernel adds
+// cross_cta_wait_offset() to the count it waits for: 0, or, for a test of
+// the error path, an offset no count ever reaches.
+constexpr unsigned long long kDefaultCrossCtaWaitNs = 1000000000ull;
+constexpr unsigned kUnreachableWaitOffset = 0x40000000u;
+unsigned long long cross_cta_wait_ns();
+unsigned cross_cta_wait_offset();
 inline cudaLaunchAttribute pdl_attribute() {
   cudaLaunchAttribute a;
   a.id = cudaLaunchAttributeProgrammaticStreamSerialization;

@@ -421,10 +421,12 @@ csa2_status run_tc(const void* q, const float* w, const void* k, int B, int Q, i
   p.n_tiles = static_cast<int>((L + kTileRows - 1) / kTileRows);
   p.n_units = static_cast<int64_t>(B) * p.n_qgroups * p.n_tiles;
   auto kern = index_tc_kernel<DK, NQ, HP, POOL>;
-  static std::once_flag once;
-  static cudaError_t attr_err = cudaSuccess;
-  std::call_once(once, [&] {
-    attr_err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::BYTES);
+  static PerDevice<cudaError_t> opt_in;
+  const cudaError_t attr_err = opt_in.get([] {
+    const cudaError_t e = cudaFuncSetAttribute(index_tc_kernel<DK, NQ, HP, POOL>,
+                                               cudaFuncAttributeMaxDynamicSharedMemorySize, C::BYTES);
+    if (e != cudaSuccess) cudaGetLastError();
+    return e;
   });
   if (attr_err != cudaSuccess) return fail(CSA2_ERR_CUDA, "index_scores_tc: smem opt-in failed");
   const int64_t grid = std::min<int64_t>(sm_count(), p.n_units);

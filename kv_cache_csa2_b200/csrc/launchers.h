@@ -25,6 +25,10 @@ csa2_status launch_index_scores(const void* q, const float* w, const void* k, in
                                 ClearOnLaunch* clear = nullptr);
 
 size_t select_topk_workspace(int64_t rows, int64_t L, int count);
+// The workspace one selection (launch_select_topk) will actually use on the
+// current device: 0 when the cluster, one-CTA or fallback kernel takes the
+// rows (select_topk_workspace is an upper bound over devices and paths).
+size_t select_topk_scratch_bytes(int64_t rows, int64_t L, int count);
 // Two selections of the same rows in one pass set (multi-CTA kernel); returns
 // CSA2_ERR_UNSUPPORTED when that kernel does not apply to the shape.
 // ws_cleared: select_topk_clear() already ran on this workspace on `stream`

@@ -721,11 +721,13 @@ csa2_status launch_variant(ClParams p, int64_t rows, cudaStream_t stream) {
   p.seg = p.chunk / NW;
   if (p.chunk > MAXCHUNK) return CSA2_ERR_UNSUPPORTED;
   using SM = Smem<NT, MAXCHUNK, SURV>;
-  static std::once_flag once;
-  static cudaError_t attr = cudaSuccess;
-  std::call_once(once, [] {
-    attr = cudaFuncSetAttribute(topk_cluster_kernel<NT, MAXCHUNK, SURV>,
-                                cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(sizeof(SM)));
+  static PerDevice<cudaError_t> opt_in;
+  const cudaError_t attr = opt_in.get([] {
+    const cudaError_t e = cudaFuncSetAttribute(topk_cluster_kernel<NT, MAXCHUNK, SURV>,
+                                               cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                               static_cast<int>(sizeof(SM)));
+    if (e != cudaSuccess) cudaGetLastError();
+    return e;
   });
   if (attr != cudaSuccess) return fail(CSA2_ERR_CUDA, "select_topk_cluster: shared-memory opt-in failed");
   cudaLaunchConfig_t cfg = {};

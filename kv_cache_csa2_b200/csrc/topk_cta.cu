@@ -464,11 +464,12 @@ csa2_status launch_select_topk_cta(const float* scores, int64_t rows, int64_t L,
   p.out[0] = out0;
   p.out[1] = out1;
   const size_t smem = smem_bytes(L, p.seg);
-  static std::once_flag once;
-  static cudaError_t attr = cudaSuccess;
-  std::call_once(once, [] {
-    attr = cudaFuncSetAttribute(topk_cta_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                static_cast<int>(smem_bytes(kSelectCtaMaxL, kSelectCtaMaxL / NW)));
+  static PerDevice<cudaError_t> opt_in;
+  const cudaError_t attr = opt_in.get([] {
+    const cudaError_t e = cudaFuncSetAttribute(topk_cta_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                               static_cast<int>(smem_bytes(kSelectCtaMaxL, kSelectCtaMaxL / NW)));
+    if (e != cudaSuccess) cudaGetLastError();
+    return e;
   });
   if (attr != cudaSuccess) return fail(CSA2_ERR_CUDA, "select_topk_cta: shared-memory opt-in failed");
   cudaLaunchConfig_t cfg = {};

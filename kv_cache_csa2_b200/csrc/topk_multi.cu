@@ -66,6 +66,8 @@ struct SelParams {
   int32_t* cpos;      // [rows][kTracks][kCandCap] their positions
   int* ccnt;          // [rows][kTracks]
   int* err;
+  unsigned long long wait_ns;   // bound of a row-barrier wait
+  unsigned wait_offset;         // added to every barrier target (0, or unreachable for tests)
 };
 
 __device__ __forceinline__ uint32_t score_key(float f) {
@@ -105,16 +107,20 @@ __device__ __forceinline__ int block_scan(int v, int* ws, int* total) {
 }
 
 // Barrier of the C CTAs working on one row: arrive on the row's counter, wait
-// (bounded: 1 s) until all have arrived `target` times in total.
-__device__ __forceinline__ bool row_barrier(unsigned* ctr, unsigned target, int* err, int* abort_s) {
+// (bounded by p.wait_ns, 1 s by default) until all have arrived `target`
+// times in total.  A CTA that gave up arrives at no later barrier and takes
+// no step that needs the other CTAs; they give up at their next barrier.
+__device__ __forceinline__ bool row_barrier(const SelParams& p, unsigned* ctr, unsigned target,
+                                            int* abort_s) {
   __syncthreads();
   if (threadIdx.x == 0 && !*abort_s) {
     __threadfence();
     atomicAdd(ctr, 1u);
     const uint64_t t0 = sm100::globaltimer_ns();
+    target += p.wait_offset;
     while (*reinterpret_cast<volatile unsigned*>(ctr) < target) {
-      if (sm100::globaltimer_ns() - t0 > 1000000000ull) {
-        raise_dev_error(err, DEVERR_TIMEOUT);
+      if (sm100::globaltimer_ns() - t0 > p.wait_ns) {
+        raise_dev_error(p.err, DEVERR_TIMEOUT);
         *abort_s = 1;
         break;
       }
@@ -231,7 +237,7 @@ __global__ void __launch_bounds__(kT, 2) topk_multi_kernel(SelParams p) {
         atomicMax(&gmm[0], ~sh_min);
         atomicMax(&gmm[1], sh_max);
       }
-      ok = row_barrier(ctr, C * (++epoch), p.err, &abort_s);
+      ok = row_barrier(p, ctr, C * (++epoch), &abort_s);
       if (tid == 0) {
         sh_min = ~__ldcg(&gmm[0]);
         sh_max = __ldcg(&gmm[1]);
@@ -274,7 +280,7 @@ __global__ void __launch_bounds__(kT, 2) topk_multi_kernel(SelParams p) {
           const int v = hist_s[t][bin];
           if (v) atomicAdd(&ghp[t * kBins + bin], v);
         }
-        ok = row_barrier(ctr, C * (++epoch), p.err, &abort_s);
+        ok = row_barrier(p, ctr, C * (++epoch), &abort_s);
         if (!ok) break;
       }
       // every CTA derives the same next prefix from the row's histogram
@@ -364,7 +370,7 @@ __global__ void __launch_bounds__(kT, 2) topk_multi_kernel(SelParams p) {
           if (tid == 0) cr[(c * kTracks + t) * 2] = tot;
         }
       }
-      ok = row_barrier(ctr, C * (++epoch), p.err, &abort_s);
+      ok = row_barrier(p, ctr, C * (++epoch), &abort_s);
       // (2) every CTA refines the threshold over the candidates (same result)
       for (int t = 0; t < p.ntracks && ok; ++t) {
         if (all[t]) continue;
@@ -544,7 +550,7 @@ __global__ void __launch_bounds__(kT, 2) topk_multi_kernel(SelParams p) {
       cr[(c * kTracks + tid) * 2] = g;
       cr[(c * kTracks + tid) * 2 + 1] = e;
     }
-    if (ok && C > 1 && !use_cand) ok = row_barrier(ctr, C * (++epoch), p.err, &abort_s);
+    if (ok && C > 1 && !use_cand) ok = row_barrier(p, ctr, C * (++epoch), &abort_s);
     __syncthreads();
     if (tid < p.ntracks && ok && !use_cand) {
       int off = 0, eq_left = need_eq[tid], take = 0, all_sel = 0;
@@ -606,26 +612,27 @@ constexpr int kChunkKeys = 8192;
 int chunk_for(int64_t L) { return L <= kOneCtaKeys ? static_cast<int>(L) : kChunkKeys; }
 
 int max_resident_ctas(size_t smem) {
-  static std::once_flag once;
-  static std::mutex mu;
-  static int per_sm_cache[2] = {-1, -1};     // [small chunk, one-CTA row]
-  std::call_once(once, [] {
+  struct PerSm {
+    int small_chunk, one_cta_row;
+  };
+  static PerDevice<PerSm> cache;
+  const PerSm per_sm = cache.get([] {
+    PerSm r{0, 0};
     if (cudaFuncSetAttribute(topk_multi_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             kOneCtaKeys * 4) != cudaSuccess)
+                             kOneCtaKeys * 4) != cudaSuccess) {
       cudaGetLastError();
-  });
-  const int slot = smem > kChunkKeys * 4 ? 1 : 0;
-  std::lock_guard<std::mutex> lk(mu);
-  if (per_sm_cache[slot] < 0) {
-    int n = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, topk_multi_kernel, kT,
-                                                      slot ? kOneCtaKeys * 4 : kChunkKeys * 4) != cudaSuccess) {
-      cudaGetLastError();
-      n = 0;
+      return r;
     }
-    per_sm_cache[slot] = n;
-  }
-  return per_sm_cache[slot] * sm_count();
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&r.small_chunk, topk_multi_kernel, kT,
+                                                      kChunkKeys * 4) != cudaSuccess ||
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&r.one_cta_row, topk_multi_kernel, kT,
+                                                      kOneCtaKeys * 4) != cudaSuccess) {
+      cudaGetLastError();
+      r = PerSm{0, 0};
+    }
+    return r;
+  });
+  return (smem > kChunkKeys * 4 ? per_sm.one_cta_row : per_sm.small_chunk) * sm_count();
 }
 
 // The one-CTA kernel of topk_cta.cu takes rows of up to kSelectCtaMaxL keys
@@ -658,6 +665,11 @@ size_t ws_bytes_for(int64_t rows, int64_t L) {
 }  // namespace
 
 size_t select_topk_multi_workspace(int64_t rows, int64_t L, int) {
+  return multi_applies(rows, L) ? ws_bytes_for(rows, L) : 0;
+}
+
+size_t select_topk_scratch_bytes(int64_t rows, int64_t L, int count) {
+  if (rows <= 0 || count <= 0 || select_topk_cluster_applies(rows, L, count, 0)) return 0;
   return multi_applies(rows, L) ? ws_bytes_for(rows, L) : 0;
 }
 
@@ -710,6 +722,8 @@ csa2_status launch_select_topk2(const float* scores, int64_t rows, int64_t L, in
   p.ckey = reinterpret_cast<uint32_t*>(static_cast<char*>(ws) + cleared + ((words * 4 + 255) & ~size_t(255)));
   p.cpos = reinterpret_cast<int32_t*>(p.ckey + rows * kTracks * kCandCap);
   p.err = device_error_word();
+  p.wait_ns = cross_cta_wait_ns();
+  p.wait_offset = cross_cta_wait_offset();
   if (C > 1 && !ws_cleared) {          // row ranges and barrier counters start at zero
     begin_launch(stream);
     if (cudaMemsetAsync(ws, 0, cleared, stream) != cudaSuccess) return check_launch("select_topk: clear");

@@ -59,7 +59,9 @@ extern "C" csa2_status csa2_select_topk_noalloc(const float* scores, int64_t row
   if (rows == 0 || count == 0) return CSA2_OK;
   if (out == nullptr || (L > 0 && scores == nullptr))
     return fail(CSA2_ERR_INVALID, "csa2_select_topk_noalloc: null pointer");
-  const size_t need = select_topk_workspace(rows, L, count);
+  // the scratch of the kernel that will run (0 for the kernels that keep
+  // their state in shared memory), not csa2_select_topk_workspace's bound
+  const size_t need = select_topk_scratch_bytes(rows, L, count);
   const size_t cap = CSA2_SELECT_TOPK_NOALLOC_SCRATCH_BYTES;
   if (need > cap)
     return fail(CSA2_ERR_OOM,

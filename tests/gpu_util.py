@@ -163,14 +163,35 @@ def oracle_group(wl, inp, sample=None):
                        n_visible=nv), new
 
 
-def compare_groups(wl, inp, gres, ores, sample=None, min_exact=0.5):
-    """Selection rule on every selecting layer; attention on the queries whose
-    selection equals the oracle's (the others differ only inside the tie band).
+def attn_on_selection(wl, kv, q_attn_bits, topk):
+    """The attention kernel, through the C ABI, on a given selection (the
+    oracle's) for the layer's queries: kv is the group's bf16 KV on the
+    device (packed to FP4 here when the workload stores FP4), q_attn_bits the
+    queries [B, Qs, Ha, D] as bf16 bits, topk int [B, Qs, k]."""
+    kv_arg, scales = kv, None
+    if wl.kv_fp4:
+        kv_arg, scales = K.csa2_fp4_pack(kv)
+    out, lse = K.csa2_sparse_attn(dev_bf16(q_attn_bits), kv_arg,
+                                  dev(np.ascontiguousarray(topk, dtype=np.int32)), wl.attn_scale,
+                                  kv_scales=scales)
+    return host_bf16(out), lse.cpu().numpy().astype(np.float64)
+
+
+def compare_groups(wl, inp, gres, ores, sample=None, min_exact=0.5, kv=None):
+    """Selection rule on every selecting layer, and attention on every layer.
+
+    Attention is checked twice.  (1) The group's own output, on the queries
+    whose selection equals the oracle's (the others differ only inside the
+    tie band); at least one query per layer, and a fraction min_exact of
+    them, must have that exact selection.  (2) When kv (the group's device
+    KV) is given, the attention kernel re-run through the C ABI on the
+    oracle's selection, for every query of the layer, against the oracle's
+    output over that selection.  Only oracle data flows into the GPU; no GPU
+    result is fed to the oracle.
 
     A Reindex layer with a pool is compared with the oracle only for queries
     whose GPU pool equals the oracle's pool; for the others the GPU row is
-    checked to be a valid subset of the GPU's own pool (no GPU data is fed to
-    the oracle)."""
+    checked to be a valid subset of the GPU's own pool."""
     sl = np.arange(wl.Q) if sample is None else np.asarray(sample)
     ik = I.bf16_bits_to_f32(inp["index_k"])
     same = np.ones((wl.B, len(sl)), dtype=bool)
@@ -207,8 +228,13 @@ def compare_groups(wl, inp, gres, ores, sample=None, min_exact=0.5):
                     if mode == "full" and wl.P > 0:
                         pool_same[b, t] = check_selection(pool_g[b, t], ids, sc, wl.P,
                                                           f"pool b{b} q{qi}")
+        assert same.any(), f"layer {i}: no query has the oracle's exact selection"
         assert same.mean() >= min_exact, f"layer {i}: only {same.mean():.2f} exact selections"
         gi = g["out"][:, sl][same]
         oi = o["o"][same]
         check_attn(gi, g["lse"][:, sl][same], oi, o["lse"][same], f"layer {i} ({mode})")
+        if kv is not None:
+            q_bits = inp["layers"][i]["q_attn"][:, sl]
+            out_r, lse_r = attn_on_selection(wl, kv, q_bits, o["topk"])
+            check_attn(out_r, lse_r, o["o"], o["lse"], f"layer {i} ({mode}) on the oracle's selection")
     return same

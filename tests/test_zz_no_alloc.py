@@ -1,8 +1,17 @@
-"""csa2_select_topk_noalloc (library-owned static scratch) against
-csa2_select_topk (caller workspace): the same selection bit for bit, on two
-calls in a row, for every path the selection takes (one CTA per row, one CTA
-per row of up to 32768 keys, several cooperating CTAs per row).  Named to be
-collected last, so it also runs after every other test in the same process."""
+"""csa2_select_topk_noalloc keeps its scratch in a static device array inside
+the library, for callers that cannot allocate device memory (for example code
+that runs while an allocator is locked, or a host runtime that hands the
+library no workspace).  Checked here against csa2_select_topk (caller
+workspace) and against the oracle's selection, on two calls in a row with new
+data each time, for every path the selection takes:
+
+  - an 8-CTA cluster per row and one CTA per row: no scratch at all;
+  - several cooperating CTAs per row (rows longer than 262144 keys, or the
+    cluster kernel switched off): the static scratch, whose counters are
+    cleared before every launch.
+
+Named to be collected last, so that it also runs after every other test in
+the same process; it needs nothing from them."""
 import ctypes
 
 import numpy as np
@@ -10,6 +19,7 @@ import pytest
 import torch
 
 import kv_cache_csa2_b200 as K
+import oracle as O
 
 CAP = 4 << 20     # CSA2_SELECT_TOPK_NOALLOC_SCRATCH_BYTES
 
@@ -21,45 +31,64 @@ def _scores(seed, rows, L, ties):
     else:
         s = r.standard_normal((rows, L)).astype(np.float32)
     s[:, ::97] = -np.inf                     # never selectable
-    return torch.from_numpy(s).cuda()
+    return s
 
 
 def _pool_ids(seed, rows, L, N):
     r = np.random.default_rng(seed)
     ids = np.stack([np.sort(r.choice(N, L, replace=False)) for _ in range(rows)]).astype(np.int32)
-    return torch.from_numpy(ids).cuda()
+    return ids
+
+
+def _oracle(s, count, ids):
+    pos = O.select_top(s.astype(np.float64), count)
+    if ids is None:
+        return pos
+    return np.where(pos >= 0, np.take_along_axis(ids, np.maximum(pos, 0), 1), -1)
 
 
 CASES = [
-    # rows, L, count, ids: one-CTA-per-row kernel (no scratch), one CTA per
-    # row (scratch, nothing cleared), cooperating CTAs (scratch, cleared)
-    (5, 1000, 64, False),
-    (8, 16384, 2048, True),
-    (8, 262144, 2048, False),
-    (3, 100000, 700, True),
+    # rows, L, count, ids, environment, uses scratch
+    (5, 1000, 64, False, {}, False),                                     # cluster of 8 CTAs
+    (64, 262144, 2048, False, {}, False),                                # cluster: rows < SMs
+    (200, 3000, 100, True, {}, False),                                   # one CTA per row
+    (5, 300000, 2048, False, {}, True),                                  # cooperating CTAs (37 per row)
+    (20, 400000, 5000, True, {}, True),                                  # 49 per row, 20 rows
+    (8, 100000, 2048, False, {"CSA2_TOPK_NO_CLUSTER": "1"}, True),       # 13 per row
 ]
 
 
 @pytest.mark.gpu
-@pytest.mark.parametrize("rows,L,count,with_ids", CASES)
-def test_noalloc_matches_workspace_entry_point(rows, L, count, with_ids):
-    assert K.lib().csa2_select_topk_workspace(rows, L, count) <= CAP
+@pytest.mark.parametrize("rows,L,count,with_ids,env,scratch", CASES)
+def test_noalloc_matches_workspace_entry_point_and_oracle(rows, L, count, with_ids, env, scratch,
+                                                          monkeypatch):
+    for k, v in env.items():
+        monkeypatch.setenv(k, v)
+    lib = K.lib()
+    ws = lib.csa2_select_topk_workspace(rows, L, count)
+    if scratch:   # the cooperative kernel runs on the static array
+        assert 0 < ws <= CAP
     for call, ties in enumerate((False, True)):           # two calls in a row, new data each
-        scores = _scores(100 + call, rows, L, ties)
+        s = _scores(100 + call, rows, L, ties)
         ids = _pool_ids(7 + call, rows, L, 4 * L) if with_ids else None
-        want = K.csa2_select_topk(scores, count, ids=ids)
-        got = K.csa2_select_topk_noalloc(scores, count, ids=ids)
-        again = K.csa2_select_topk_noalloc(scores, count, ids=ids)
+        ds = torch.from_numpy(s).cuda()
+        di = torch.from_numpy(ids).cuda() if ids is not None else None
+        want = K.csa2_select_topk(ds, count, ids=di)
+        got = K.csa2_select_topk_noalloc(ds, count, ids=di)
+        again = K.csa2_select_topk_noalloc(ds, count, ids=di)
         torch.cuda.synchronize()
         assert torch.equal(got, want)
         assert torch.equal(again, want)
+        assert np.array_equal(got.cpu().numpy(), _oracle(s, count, ids))
     K.csa2_device_error()
 
 
 def test_noalloc_rejects_oversize_on_host():
-    """More rows than the static scratch holds: CSA2_ERR_OOM, nothing enqueued."""
+    """A cooperative selection whose scratch exceeds the static array:
+    CSA2_ERR_OOM with nothing enqueued (26 rows of 400000 keys need about
+    4.3 MiB; 25 rows is the most the array holds on that path)."""
     lib = K.lib()
-    rows, L, count = 64, 262144, 2048
+    rows, L, count = 26, 400000, 2048
     need = lib.csa2_select_topk_workspace(rows, L, count)
     assert need > CAP
     p = ctypes.c_void_p(256)
@@ -67,5 +96,6 @@ def test_noalloc_rejects_oversize_on_host():
     assert st == 6
     msg = lib.csa2_last_error().decode()
     assert str(need) in msg and str(CAP) in msg
+    assert lib.csa2_select_topk_workspace(25, L, count) <= CAP
     # empty work needs no scratch
     assert lib.csa2_select_topk_noalloc(None, 0, L, count, None, None, None) == 0
