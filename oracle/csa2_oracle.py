@@ -26,7 +26,8 @@ named in the function's docstring):
 Pinning status (what checks this file against something other than itself is
 listed in tests/test_oracle_pins.py):
   bf16 rounding, compression, index score, top-k / pool, attention, FP4
-  pack/unpack, and the three layer modes are all pinned.  The pages' model-level
+  pack/unpack, the three layer modes, the sliding-window branch and its
+  merge, HCA compression and HCA (dense) attention are all pinned.  The pages' model-level
   figures (about 890 bytes per token, 437x smaller than V1) are "parity
   unpinned": they cannot be derived from the pages.
 """
@@ -264,6 +265,128 @@ def sparse_attn(q: np.ndarray, kv: np.ndarray, topk: np.ndarray, scale: float):
 
 
 # ----------------------------------------------------------------------------
+# sliding-window branch and its merge with the CSA2 branch
+# ----------------------------------------------------------------------------
+
+
+def swa_attn(q: np.ndarray, win: np.ndarray, win_end: np.ndarray, W: int, scale: float):
+    """The sliding-window attention branch of a layer (V4.1 Flash transcript,
+    the paragraph on the layer layout: every CSA2 layer keeps a sliding-window
+    attention branch over its own, uncompressed KV of the most recent 128
+    tokens).  Readings: the window rows are attended like the compressed
+    entries of eq. 9 (the same query heads and scale, the row serving as key
+    and value); query (b, t) takes rows [max(0, e - W), e) of sequence b's
+    window buffer with e = win_end[b, t].
+
+    Args: q [B, Q, Ha, D]; win [B, R, D] row values; win_end int [B, Q].
+    Returns (o [B, Q, Ha, D], lse [B, Q, Ha]) float64; an empty window gives
+    o = 0, lse = -inf.
+    """
+    q = np.asarray(q, dtype=np.float64)
+    win = np.asarray(win, dtype=np.float64)
+    B, Q, Ha, D = q.shape
+    o = np.zeros((B, Q, Ha, D), dtype=np.float64)
+    lse = np.full((B, Q, Ha), -np.inf, dtype=np.float64)
+    for b in range(B):
+        for t in range(Q):
+            e = int(win_end[b, t])
+            rows = win[b, max(0, e - W):e]
+            if rows.shape[0] == 0:
+                continue
+            logits = scale * (q[b, t] @ rows.T)       # [Ha, w]
+            top = logits.max(axis=1, keepdims=True)
+            p = np.exp(logits - top)
+            l = p.sum(axis=1, keepdims=True)
+            o[b, t] = (p @ rows) / l
+            lse[b, t] = (top + np.log(l))[:, 0]
+    return o, lse
+
+
+def lse_merge(o1: np.ndarray, lse1: np.ndarray, o2: np.ndarray, lse2: np.ndarray):
+    """Combine two attention branches that were each normalised over their own
+    rows into the result of one softmax over the union of their rows: each
+    branch is weighted by its share exp(lse_i) of the total mass.  A branch
+    with lse = -inf (no rows) has no weight.  Returns (o, lse) float64."""
+    lse1 = np.asarray(lse1, dtype=np.float64)
+    lse2 = np.asarray(lse2, dtype=np.float64)
+    top = np.maximum(lse1, lse2)
+    safe = np.where(np.isfinite(top), top, 0.0)
+    w1 = np.where(np.isfinite(lse1), np.exp(lse1 - safe), 0.0)
+    w2 = np.where(np.isfinite(lse2), np.exp(lse2 - safe), 0.0)
+    tot = w1 + w2
+    den = np.where(tot > 0, tot, 1.0)
+    o = (w1[..., None] * np.asarray(o1, dtype=np.float64) +
+         w2[..., None] * np.asarray(o2, dtype=np.float64)) / den[..., None]
+    lse = np.where(tot > 0, safe + np.log(den), -np.inf)
+    return o, lse
+
+
+def sparse_attn_swa(q, kv, topk, win, win_end, W: int, scale: float):
+    """A CSA2 layer's attention with its sliding-window branch: the CSA2 branch
+    over the selected entries (sparse_attn) merged with the window branch
+    (swa_attn) by lse_merge.  Returns (o_exact, o_bf16, lse)."""
+    o1, _, l1 = sparse_attn(q, kv, topk, scale)
+    o2, l2 = swa_attn(q, win, win_end, W, scale)
+    o, lse = lse_merge(o1, l1, o2, l2)
+    return o, round_to_bf16(o), lse
+
+
+# ----------------------------------------------------------------------------
+# HCA: no-overlap compression and attention over every entry
+# ----------------------------------------------------------------------------
+
+
+def compress_hca(c: np.ndarray, z: np.ndarray, bias: np.ndarray, m: int):
+    """HCA compression (V4 explainer, HCA 压缩机制, eq. 10; weights as eq. 11):
+    like CSA's, but over larger groups of m tokens and without joining two
+    consecutive groups, so entry j is the per-channel softmax (logits z plus
+    the bias of the position inside the group) weighted sum of the values c of
+    tokens [j m, (j+1) m).  bias: [m, D].  A trailing partial group forms no
+    entry.  Returns (e_exact, e_bf16) float64 [B, T // m, D]."""
+    c = np.asarray(c, dtype=np.float64)
+    z = np.asarray(z, dtype=np.float64)
+    bias = np.asarray(bias, dtype=np.float64)
+    assert bias.shape[0] == m
+    B, T, D = c.shape
+    N = T // m
+    e = np.zeros((B, N, D), dtype=np.float64)
+    for j in range(N):
+        rows = slice(j * m, (j + 1) * m)
+        logits = z[:, rows, :] + bias[None, :, :]
+        top = logits.max(axis=1, keepdims=True)
+        p = np.exp(logits - top)
+        p /= p.sum(axis=1, keepdims=True)
+        e[:, j, :] = (p * c[:, rows, :]).sum(axis=1)
+    return e, round_to_bf16(e)
+
+
+def dense_attn(q: np.ndarray, kv: np.ndarray, scale: float, n_visible=None):
+    """HCA attention (V4 explainer, HCA 注意力计算): eq. 9's shared-KV attention
+    over every compressed entry, no selection.  Query (b, t) takes entries
+    [0, n_visible[b, t]) (all when n_visible is None).
+    Returns (o_exact, o_bf16, lse) float64."""
+    q = np.asarray(q, dtype=np.float64)
+    kv = np.asarray(kv, dtype=np.float64)
+    B, Q, Ha, D = q.shape
+    N = kv.shape[1]
+    o = np.zeros((B, Q, Ha, D), dtype=np.float64)
+    lse = np.full((B, Q, Ha), -np.inf, dtype=np.float64)
+    for b in range(B):
+        for t in range(Q):
+            n = N if n_visible is None else min(N, int(n_visible[b, t]))
+            if n <= 0:
+                continue
+            ent = kv[b, :n]
+            logits = scale * (q[b, t] @ ent.T)
+            top = logits.max(axis=1, keepdims=True)
+            p = np.exp(logits - top)
+            l = p.sum(axis=1, keepdims=True)
+            o[b, t] = (p @ ent) / l
+            lse[b, t] = (top + np.log(l))[:, 0]
+    return o, round_to_bf16(o), lse
+
+
+# ----------------------------------------------------------------------------
 # (a5) FP4 main-KV format: E2M1 values, one E4M3 scale per 16 channels
 # ----------------------------------------------------------------------------
 
@@ -383,7 +506,9 @@ def run_group(modes, layers, kv, index_k, k_top: int, scale: float,
 
     kv: [B, N, D] main-KV values (already dequantised when stored as FP4), or
     a row-fetch function kv(b, ids) as sparse_attn takes; index_k: [B, N, d].  layers[i] holds 'q_attn' and, for full/reindex,
-    'q_index' and 'w_index'.  Returns a list of per-layer dicts with
+    'q_index' and 'w_index', and optionally 'swa' = (win, win_end, W), the
+    layer's sliding-window rows (attention then merges that branch, see
+    sparse_attn_swa).  Returns a list of per-layer dicts with
     'topk', 'pool' (full only), 'o' (exact), 'o_bf16', 'lse'.
     """
     results = []
@@ -415,7 +540,11 @@ def run_group(modes, layers, kv, index_k, k_top: int, scale: float,
                 raise ValueError("reuse before any full layer")
         else:
             raise ValueError(mode)
-        o, o16, lse = sparse_attn(L["q_attn"], kv, topk, scale)
+        if L.get("swa") is not None:          # the layer's own sliding-window branch
+            win, win_end, W = L["swa"]
+            o, o16, lse = sparse_attn_swa(L["q_attn"], kv, topk, win, win_end, W, scale)
+        else:
+            o, o16, lse = sparse_attn(L["q_attn"], kv, topk, scale)
         res.update(topk=topk, o=o, o_bf16=o16, lse=lse)
         results.append(res)
     return results
