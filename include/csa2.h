@@ -102,6 +102,18 @@ csa2_status csa2_compress(const void* c, const float* z, const float* bias, int 
                           int D, int m, int has_left_halo, void* out, int64_t out_batch_stride,
                           csa2_stream stream);
 
+/* HCA (heavily compressed attention) compression.  [V4] HCA 压缩机制, eq. (10)
+ * with the weights of eq. (11): blocks of m tokens (m >> the CSA block), and
+ * unlike csa2_compress an entry does not join two consecutive blocks:
+ *   e[b, j, ch] = sum_{t in [jm, (j+1)m)} softmax_t(z[b,t,ch] + bias[t - jm, ch]) * c[b,t,ch]
+ * f32 arithmetic (one pass with a running max), rounded once to bf16.
+ *   c bf16 [B, T, D]    z f32 [B, T, D]    bias f32 [m, D]
+ *   out bf16 entries j in [0, T/m) at out + b*out_batch_stride + j*D (stride 0 = (T/m)*D).
+ * Requires D % 8 == 0, 1 <= m <= 1024.  Errors: CSA2_ERR_INVALID. */
+csa2_status csa2_compress_hca(const void* c, const float* z, const float* bias, int B, int64_t T,
+                              int D, int m, void* out, int64_t out_batch_stride,
+                              csa2_stream stream);
+
 /* ------------------------------------------------------------------------ */
 /* (a2) Lightning-indexer scores.  [V4] 闪电索引机制, eq. (8):
  *   s[b,q,j] = sum_h w[b,q,h] * act(q[b,q,h,:] . k[b,e,:])
@@ -209,6 +221,41 @@ csa2_status csa2_sparse_attn(csa2_mode mode, const void* q, const csa2_kv* kv,
                              void* out, float* lse, void* workspace, size_t workspace_bytes,
                              csa2_stream stream);
 
+/* (a4 + SWA branch) Sparse attention together with the layer's sliding-window
+ * branch.  [V41] layer layout: every CSA2 layer keeps a sliding-window
+ * attention branch over its own uncompressed KV of the most recent 128 tokens
+ * (layer-specific, never shared between layers).  Reading: the window rows
+ * enter the same softmax as the selected entries (same heads, same scale,
+ * shared K = V), which equals merging the two branches' normalised outputs by
+ * their log-sum-exp: out = (e^lse_c out_c + e^lse_w out_w) / (e^lse_c + e^lse_w),
+ * lse = log(e^lse_c + e^lse_w).  The kernel merges f32 partials, not rounded
+ * branch outputs.
+ *   win     bf16 [B, win_rows, D]: each sequence's uncompressed window rows
+ *   win_end int32 [B, Q]: query (b, q) attends rows [max(0, e - W), e) of
+ *           sequence b with e = win_end[b, q], 0 <= e <= win_rows (decode: the
+ *           last W rows with e = win_rows; a prefill chunk: e = the query's
+ *           own row + 1)
+ *   W       window length, 1 <= W <= 128
+ * Other arguments, outputs and errors are csa2_sparse_attn's; an e outside
+ * [0, win_rows] is recorded as CSA2_ERR_BOUNDS and the window taken empty.
+ * workspace: csa2_sparse_attn_swa_workspace(...) bytes. */
+size_t csa2_sparse_attn_swa_workspace(int B, int Q, int Ha, int D, int k, csa2_kv_fmt fmt);
+csa2_status csa2_sparse_attn_swa(csa2_mode mode, const void* q, const csa2_kv* kv,
+                                 const int32_t* topk, int B, int Q, int Ha, int k, float scale,
+                                 const void* win, int64_t win_rows, const int32_t* win_end, int W,
+                                 void* out, float* lse, void* workspace, size_t workspace_bytes,
+                                 csa2_stream stream);
+
+/* HCA attention.  [V4] HCA 注意力计算: the queries attend, as in eq. (9) with
+ * shared K = V, to every compressed entry (no indexer, no top-k).  Query
+ * (b, q) takes entries [0, n_visible[b, q]) of sequence b (n_visible = NULL:
+ * all kv->n).  Same kernels, outputs and errors as csa2_sparse_attn with the
+ * selection j -> j.  workspace: csa2_dense_attn_workspace(B, Q, Ha, D, kv->n, fmt). */
+size_t csa2_dense_attn_workspace(int B, int Q, int Ha, int D, int64_t N, csa2_kv_fmt fmt);
+csa2_status csa2_dense_attn(const void* q, const csa2_kv* kv, const int32_t* n_visible, int B,
+                            int Q, int Ha, float scale, void* out, float* lse, void* workspace,
+                            size_t workspace_bytes, csa2_stream stream);
+
 /* ------------------------------------------------------------------------ */
 /* (a5) FP4 main-KV format.  [R] FP4 主KV缓存: E2M1 with one E4M3 scale per 16
  * channels.  Per 16-channel block: scale s = E4M3 value nearest absmax/6
@@ -265,6 +312,12 @@ typedef struct {
   const void* q_attn;        /* all modes: bf16 [B, Q, Ha, D]                               */
   void* out;                 /* all modes: bf16 [B, Q, Ha, D]                               */
   float* lse;                /* all modes: f32 [B, Q, Ha] or NULL                           */
+  /* Optional sliding-window branch of this layer (csa2_sparse_attn_swa):
+   * NULL swa_kv = none.  Each layer passes its own window rows. */
+  const void* swa_kv;        /* bf16 [B, swa_rows, D]                                        */
+  int64_t swa_rows;
+  const int32_t* swa_end;    /* int32 [B, Q]                                                 */
+  int swa_window;            /* W, 1..128                                                    */
 } csa2_layer_io;
 
 csa2_status csa2_group_create(csa2_group** group, const csa2_group_desc* desc);

@@ -14,7 +14,8 @@ __all__ = [
     "CSA2Error", "lib", "lib_path", "FULL", "REINDEX", "REUSE", "KV_BF16", "KV_FP4", "ACT_RELU",
     "ACT_IDENTITY", "csa2_compress", "csa2_index_scores", "csa2_select_topk", "csa2_select_topk_noalloc",
     "csa2_index_topk",
-    "csa2_sparse_attn", "csa2_fp4_pack", "csa2_fp4_unpack", "Group", "csa2_device_error",
+    "csa2_sparse_attn", "csa2_sparse_attn_swa", "csa2_dense_attn", "csa2_compress_hca",
+    "csa2_fp4_pack", "csa2_fp4_unpack", "Group", "csa2_device_error",
     "launch_counts", "reset_launch_counts", "set_fault", "set_device_wait", "EXPORTED_SYMBOLS",
 ]
 
@@ -39,7 +40,8 @@ class CSA2GroupDesc(ctypes.Structure):
 
 class CSA2LayerIO(ctypes.Structure):
     _fields_ = [("kv", CSA2Kv), ("index_k", _P), ("n_visible", _P), ("q_index", _P),
-                ("w_index", _P), ("q_attn", _P), ("out", _P), ("lse", _P)]
+                ("w_index", _P), ("q_attn", _P), ("out", _P), ("lse", _P),
+                ("swa_kv", _P), ("swa_rows", _I64), ("swa_end", _P), ("swa_window", _I)]
 
 
 # name -> (restype, argtypes); every symbol include/csa2.h declares
@@ -55,6 +57,12 @@ _SIGS = {
     "csa2_sparse_attn_workspace": (_SZ, [_I, _I, _I, _I, _I, _I]),
     "csa2_sparse_attn": (_I, [_I, _P, ctypes.POINTER(CSA2Kv), _P, _I, _I, _I, _I, _F, _P, _P, _P,
                               _SZ, _P]),
+    "csa2_sparse_attn_swa_workspace": (_SZ, [_I, _I, _I, _I, _I, _I]),
+    "csa2_sparse_attn_swa": (_I, [_I, _P, ctypes.POINTER(CSA2Kv), _P, _I, _I, _I, _I, _F, _P, _I64,
+                                  _P, _I, _P, _P, _P, _SZ, _P]),
+    "csa2_dense_attn_workspace": (_SZ, [_I, _I, _I, _I, _I64, _I]),
+    "csa2_dense_attn": (_I, [_P, ctypes.POINTER(CSA2Kv), _P, _I, _I, _I, _F, _P, _P, _P, _SZ, _P]),
+    "csa2_compress_hca": (_I, [_P, _P, _P, _I, _I64, _I, _I, _P, _I64, _P]),
     "csa2_fp4_pack": (_I, [_P, _I64, _I, _P, _P, _P]),
     "csa2_fp4_unpack": (_I, [_P, _P, _I64, _I, _P, _P]),
     "csa2_group_create": (_I, [ctypes.POINTER(_P), ctypes.POINTER(CSA2GroupDesc)]),
@@ -252,6 +260,64 @@ def csa2_sparse_attn(q, kv, topk, scale: float, kv_scales=None, mode=FULL, out=N
     return out, lse
 
 
+def csa2_sparse_attn_swa(q, kv, topk, scale: float, win, win_end, W: int = 128, kv_scales=None,
+                         mode=FULL, out=None, lse=None, stream=None):
+    """Sparse attention with the layer's sliding-window branch in the same
+    softmax: win bf16 [B, R, D] window rows, win_end int32 [B, Q]."""
+    torch = _torch()
+    _need(q, torch.bfloat16, 4, "q")
+    _need(topk, torch.int32, 3, "topk")
+    _need(win, torch.bfloat16, 3, "win")
+    _need(win_end, torch.int32, 2, "win_end")
+    B, Q, Ha, D = q.shape
+    k = topk.shape[2]
+    desc = make_kv(kv, kv_scales)
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty(B, Q, Ha, dtype=torch.float32, device=q.device)
+    nb = lib().csa2_sparse_attn_swa_workspace(B, Q, Ha, D, k, desc.fmt)
+    ws = _workspace(nb, q.device)
+    _check(lib().csa2_sparse_attn_swa(_MODE[mode], _ptr(q), ctypes.byref(desc), _ptr(topk), B, Q,
+                                      Ha, k, scale, _ptr(win), win.shape[1], _ptr(win_end), W,
+                                      _ptr(out), _ptr(lse), _ptr(ws), nb, _stream(stream)))
+    return out, lse
+
+
+def csa2_dense_attn(q, kv, scale: float, n_visible=None, kv_scales=None, out=None, lse=None,
+                    stream=None):
+    """HCA attention: every query attends to entries [0, n_visible) of its sequence."""
+    torch = _torch()
+    _need(q, torch.bfloat16, 4, "q")
+    if n_visible is not None:
+        _need(n_visible, torch.int32, 2, "n_visible")
+    B, Q, Ha, D = q.shape
+    desc = make_kv(kv, kv_scales)
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty(B, Q, Ha, dtype=torch.float32, device=q.device)
+    nb = lib().csa2_dense_attn_workspace(B, Q, Ha, D, desc.n, desc.fmt)
+    ws = _workspace(nb, q.device)
+    _check(lib().csa2_dense_attn(_ptr(q), ctypes.byref(desc), _ptr(n_visible), B, Q, Ha, scale,
+                                 _ptr(out), _ptr(lse), _ptr(ws), nb, _stream(stream)))
+    return out, lse
+
+
+def csa2_compress_hca(c, z, bias, m: int, out=None, out_batch_stride: int = 0, stream=None):
+    """HCA compression of raw tokens (c bf16 / z f32 [B, T, D], bias f32 [m, D])."""
+    torch = _torch()
+    _need(c, torch.bfloat16, 3, "c")
+    _need(z, torch.float32, 3, "z")
+    _need(bias, torch.float32, 2, "bias")
+    B, T, D = c.shape
+    if out is None:
+        out = torch.empty(B, T // m, D, dtype=torch.bfloat16, device=c.device)
+    _check(lib().csa2_compress_hca(_ptr(c), _ptr(z), _ptr(bias), B, T, D, m, _ptr(out),
+                                   out_batch_stride, _stream(stream)))
+    return out
+
+
 # ------------------------------------------------------------------ (a5)
 def csa2_fp4_pack(x, stream=None):
     torch = _torch()
@@ -289,7 +355,9 @@ class Group:
         self.desc = desc
 
     def layer(self, i, q_attn, out, lse=None, kv=None, kv_scales=None, index_k=None,
-              q_index=None, w_index=None, n_visible=None, stream=None):
+              q_index=None, w_index=None, n_visible=None, swa=None, stream=None):
+        """swa: optional (win bf16 [B, R, D], win_end int32 [B, Q], W), this
+        layer's own sliding-window rows."""
         io = CSA2LayerIO()
         if kv is not None:
             io.kv = make_kv(kv, kv_scales)
@@ -300,6 +368,12 @@ class Group:
         io.q_attn = _ptr(q_attn)
         io.out = _ptr(out)
         io.lse = _ptr(lse)
+        if swa is not None:
+            win, win_end, W = swa
+            io.swa_kv = _ptr(win)
+            io.swa_rows = win.shape[1]
+            io.swa_end = _ptr(win_end)
+            io.swa_window = W
         _check(lib().csa2_group_layer(self._h, i, ctypes.byref(io), _stream(stream)))
 
     def selection(self):

@@ -193,7 +193,8 @@ namespace csa2 {
 csa2_status sparse_attn_checked(csa2_mode mode, const void* q, const csa2_kv* kv,
                                 const int32_t* topk, int B, int Q, int Ha, int k, float scale,
                                 void* out, float* lse, void* workspace, size_t workspace_bytes,
-                                unsigned long long* sync_zeroed, cudaStream_t stream) {
+                                unsigned long long* sync_zeroed, cudaStream_t stream,
+                                const AttnRows& rows) {
   CSA2_TRY(fault_gate());
   REQUIRE(mode == CSA2_FULL || mode == CSA2_REINDEX || mode == CSA2_REUSE,
           "csa2_sparse_attn: unknown mode %d", int(mode));
@@ -204,13 +205,18 @@ csa2_status sparse_attn_checked(csa2_mode mode, const void* q, const csa2_kv* kv
   REQUIRE(kv->n >= 0 && kv->n <= 0x7fffffffLL, "csa2_sparse_attn: bad kv->n");
   if (B == 0 || Q == 0) return CSA2_OK;
   REQUIRE_PTR(q); REQUIRE_PTR(out); REQUIRE_PTR(kv->data);
-  REQUIRE(k == 0 || topk != nullptr, "csa2_sparse_attn: topk is null");
   REQUIRE(kv->fmt == CSA2_KV_BF16 || kv->scales != nullptr, "csa2_sparse_attn: FP4 kv without scales");
-  const size_t need = sparse_attn_workspace(B, Q, Ha, kv->dim, k, kv->fmt);
+  if (rows.win) {
+    REQUIRE(aligned16(rows.win) && rows.win_end != nullptr && rows.win_rows >= 0 &&
+                rows.win_rows <= 0x7fffffffLL && rows.W >= 1 && rows.W <= kMaxWindow,
+            "csa2_sparse_attn: window rows need a 16-byte aligned buffer, win_end and 1 <= W <= %d",
+            kMaxWindow);
+  }
+  const size_t need = sparse_attn_workspace(B, Q, Ha, kv->dim, k, kv->fmt, rows.win != nullptr);
   if (workspace_bytes < need || (need > 0 && !workspace))
     return fail(CSA2_ERR_OOM, "csa2_sparse_attn: workspace %zu < %zu bytes", workspace_bytes, need);
   return launch_sparse_attn(q, *kv, topk, B, Q, Ha, k, scale, out, lse, workspace, workspace_bytes,
-                            sync_zeroed, stream);
+                            sync_zeroed, stream, rows);
 }
 }  // namespace csa2
 
@@ -233,7 +239,7 @@ const char* csa2_status_string(csa2_status s) {
 
 const char* csa2_last_error(void) { return t_msg; }
 
-int csa2_version(void) { return 1; }
+int csa2_version(void) { return 2; }
 
 csa2_status csa2_set_device_wait(uint64_t limit_ns, int unreachable) {
   g_wait_ns.store(limit_ns);
@@ -333,6 +339,24 @@ csa2_status csa2_compress(const void* c, const float* z, const float* bias, int 
           (long long)out_batch_stride);
   return launch_compress(c, z, bias, B, T, D, m, has_left_halo ? 1 : 0, out, out_batch_stride,
                          reinterpret_cast<cudaStream_t>(stream));
+}
+
+csa2_status csa2_compress_hca(const void* c, const float* z, const float* bias, int B, int64_t T,
+                              int D, int m, void* out, int64_t out_batch_stride,
+                              csa2_stream stream) {
+  CSA2_TRY(fault_gate());
+  REQUIRE(B >= 0 && T >= 0, "csa2_compress_hca: negative size (B=%d, T=%lld)", B, (long long)T);
+  REQUIRE(D > 0 && D % 8 == 0, "csa2_compress_hca: D=%d must be a positive multiple of 8", D);
+  REQUIRE(m >= 1 && m <= kMaxHcaBlock, "csa2_compress_hca: m=%d outside [1, %d]", m, kMaxHcaBlock);
+  const int64_t N = T / m;
+  if (B == 0 || N == 0) return CSA2_OK;
+  REQUIRE_PTR(c); REQUIRE_PTR(z); REQUIRE_PTR(bias); REQUIRE_PTR(out);
+  if (out_batch_stride == 0) out_batch_stride = N * D;
+  REQUIRE(out_batch_stride >= N * D && out_batch_stride % 8 == 0,
+          "csa2_compress_hca: out_batch_stride=%lld must be >= (T/m)*D and a multiple of 8",
+          (long long)out_batch_stride);
+  return launch_compress_hca(c, z, bias, B, T, D, m, out, out_batch_stride,
+                             reinterpret_cast<cudaStream_t>(stream));
 }
 
 // ------------------------------------------------------------- (a2)
@@ -452,8 +476,46 @@ csa2_status csa2_sparse_attn(csa2_mode mode, const void* q, const csa2_kv* kv,
                              const int32_t* topk, int B, int Q, int Ha, int k, float scale,
                              void* out, float* lse, void* workspace, size_t workspace_bytes,
                              csa2_stream stream) {
+  REQUIRE(k <= 0 || B <= 0 || Q <= 0 || topk != nullptr, "csa2_sparse_attn: topk is null");
   return sparse_attn_checked(mode, q, kv, topk, B, Q, Ha, k, scale, out, lse, workspace,
                              workspace_bytes, nullptr, reinterpret_cast<cudaStream_t>(stream));
+}
+
+size_t csa2_sparse_attn_swa_workspace(int B, int Q, int Ha, int D, int k, csa2_kv_fmt fmt) {
+  return sparse_attn_workspace(B, Q, Ha, D, k, fmt, true);
+}
+
+csa2_status csa2_sparse_attn_swa(csa2_mode mode, const void* q, const csa2_kv* kv,
+                                 const int32_t* topk, int B, int Q, int Ha, int k, float scale,
+                                 const void* win, int64_t win_rows, const int32_t* win_end, int W,
+                                 void* out, float* lse, void* workspace, size_t workspace_bytes,
+                                 csa2_stream stream) {
+  REQUIRE(k <= 0 || B <= 0 || Q <= 0 || topk != nullptr, "csa2_sparse_attn_swa: topk is null");
+  REQUIRE(win != nullptr, "csa2_sparse_attn_swa: window rows are null");
+  AttnRows rows;
+  rows.win = win;
+  rows.win_rows = win_rows;
+  rows.win_end = win_end;
+  rows.W = W;
+  return sparse_attn_checked(mode, q, kv, topk, B, Q, Ha, k, scale, out, lse, workspace,
+                             workspace_bytes, nullptr, reinterpret_cast<cudaStream_t>(stream), rows);
+}
+
+size_t csa2_dense_attn_workspace(int B, int Q, int Ha, int D, int64_t N, csa2_kv_fmt fmt) {
+  if (N < 0 || N > 0x7fffffffLL) return 0;
+  return sparse_attn_workspace(B, Q, Ha, D, static_cast<int>(N), fmt, false);
+}
+
+csa2_status csa2_dense_attn(const void* q, const csa2_kv* kv, const int32_t* n_visible, int B,
+                            int Q, int Ha, float scale, void* out, float* lse, void* workspace,
+                            size_t workspace_bytes, csa2_stream stream) {
+  REQUIRE(kv != nullptr, "csa2_dense_attn: kv is null");
+  REQUIRE(kv->n >= 0 && kv->n <= 0x7fffffffLL, "csa2_dense_attn: bad kv->n");
+  AttnRows rows;
+  rows.n_visible = n_visible;
+  return sparse_attn_checked(CSA2_FULL, q, kv, nullptr, B, Q, Ha, static_cast<int>(kv->n), scale,
+                             out, lse, workspace, workspace_bytes, nullptr,
+                             reinterpret_cast<cudaStream_t>(stream), rows);
 }
 
 // ------------------------------------------------------------- (a5)

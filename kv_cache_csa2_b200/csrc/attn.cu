@@ -18,8 +18,8 @@ namespace csa2 {
 csa2_status launch_sparse_attn_tc(const void* q, const csa2_kv& kv, const int32_t* topk, int B,
                                   int Q, int Ha, int k, float scale, void* out, float* lse,
                                   void* ws, size_t ws_bytes, unsigned long long* sync_zeroed,
-                                  cudaStream_t stream);
-size_t sparse_attn_tc_workspace(int B, int Q, int Ha, int D, int k, csa2_kv_fmt fmt);
+                                  cudaStream_t stream, const AttnRows& rows);
+size_t sparse_attn_tc_workspace(int B, int Q, int Ha, int D, int k, csa2_kv_fmt fmt, bool win);
 
 namespace {
 
@@ -31,14 +31,23 @@ struct AttnSmem {
   static constexpr int RS = DD + 1;  // padded f32 row stride: conflict-free column reads
   static constexpr size_t q_words = HA * DD / 2;
   static constexpr size_t bytes = q_words * 4 + size_t(kR) * RS * 4 + size_t(HA) * (kR + 1) * 4 +
-                                  3 * HA * 4 + kR * 4;
+                                  3 * HA * 4 + 2 * kR * 4;
+};
+
+// The row sources of launch_sparse_attn (AttnRows) as the kernel takes them.
+struct SimtRows {
+  const int32_t* n_visible;
+  const uint16_t* win;
+  int64_t win_rows;
+  const int32_t* win_end;
+  int W;
 };
 
 template <int HA, int DD, bool FP4>
 __global__ void __launch_bounds__(kT) attn_simt_kernel(
     const uint16_t* __restrict__ q, const void* __restrict__ kv_data,
     const uint8_t* __restrict__ kv_scales, int64_t n, const int32_t* __restrict__ topk, int k,
-    float scale, uint16_t* __restrict__ out, float* __restrict__ lse, int* err) {
+    float scale, uint16_t* __restrict__ out, float* __restrict__ lse, int* err, SimtRows rs) {
   using S = AttnSmem<HA, DD>;
   constexpr int TPH = kT / HA;      // threads per head in the accumulation
   constexpr int OPT = DD / TPH;     // outputs per thread
@@ -51,7 +60,8 @@ __global__ void __launch_bounds__(kT) attn_simt_kernel(
   float* m_s = p_s + HA * (kR + 1);
   float* l_s = m_s + HA;
   float* a_s = l_s + HA;
-  int* id_s = reinterpret_cast<int*>(a_s + HA);
+  int* id_s = reinterpret_cast<int*>(a_s + HA);   // [kR] row ids; [kR] their source (1 = window)
+  int* src_s = id_s + kR;
 
   const int tid = threadIdx.x;
   const int64_t seq = blockIdx.y;                                   // sequence b
@@ -63,14 +73,38 @@ __global__ void __launch_bounds__(kT) attn_simt_kernel(
   float acc[OPT];
 #pragma unroll
   for (int i = 0; i < OPT; ++i) acc[i] = 0.0f;
-  const int32_t* ids = topk + qi * k;
+  // slots: k selected (topk, or dense: slot j is entry j while j < n_visible),
+  // then W window rows
+  const int64_t vis = (!topk && rs.n_visible) ? rs.n_visible[qi] : k;
+  int w_end = 0;
+  if (rs.win) {
+    w_end = rs.win_end[qi];
+    if (w_end < 0 || w_end > rs.win_rows) {
+      if (tid == 0) raise_dev_error(err, DEVERR_BOUNDS);
+      w_end = 0;
+    }
+  }
+  const int slots = k + (rs.win ? rs.W : 0);
 
-  for (int c0 = 0; c0 < k; c0 += kR) {
+  for (int c0 = 0; c0 < slots; c0 += kR) {
     __syncthreads();   // previous step done with rows_s / p_s / id_s
     if (tid < kR) {
-      int id = (c0 + tid < k) ? ids[c0 + tid] : -1;
-      if (id >= n || id < -1) { raise_dev_error(err, DEVERR_BOUNDS); id = -1; }
+      const int s = c0 + tid;
+      int id = -1, src = 0;
+      if (s < k) {
+        if (topk) {
+          id = topk[qi * k + s];
+          if (id >= n || id < -1) { raise_dev_error(err, DEVERR_BOUNDS); id = -1; }
+        } else {
+          id = s < vis ? s : -1;
+        }
+      } else if (s < slots) {
+        const int row = w_end - rs.W + (s - k);
+        id = row >= 0 ? row : -1;
+        src = 1;
+      }
       id_s[tid] = id;
+      src_s[tid] = src;
     }
     __syncthreads();
     // stage rows as f32 (zeros for empty slots)
@@ -80,9 +114,11 @@ __global__ void __launch_bounds__(kT) attn_simt_kernel(
         const int r = i / V, c = i % V;
         const int id = id_s[r];
         uint4 v = make_uint4(0, 0, 0, 0);
-        if (id >= 0)
-          v = __ldg(reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(kv_data) +
-                                                   (seq * n + id) * DD) + c);
+        if (id >= 0) {
+          const uint16_t* base = src_s[r] ? rs.win + (seq * rs.win_rows + id) * DD
+                                          : static_cast<const uint16_t*>(kv_data) + (seq * n + id) * DD;
+          v = __ldg(reinterpret_cast<const uint4*>(base) + c);
+        }
         float* dst = rows_s + r * S::RS + c * 8;
         dst[0] = bf16_lo(v.x); dst[1] = bf16_hi(v.x); dst[2] = bf16_lo(v.y); dst[3] = bf16_hi(v.y);
         dst[4] = bf16_lo(v.z); dst[5] = bf16_hi(v.z); dst[6] = bf16_lo(v.w); dst[7] = bf16_hi(v.w);
@@ -96,6 +132,17 @@ __global__ void __launch_bounds__(kT) attn_simt_kernel(
         if (id < 0) {
 #pragma unroll
           for (int u = 0; u < 16; ++u) dst[u] = 0.0f;
+          continue;
+        }
+        if (src_s[r]) {            // window rows are uncompressed bf16
+          const uint4* wp = reinterpret_cast<const uint4*>(rs.win + (seq * rs.win_rows + id) * DD + blk * 16);
+          const uint4 a = __ldg(wp), b = __ldg(wp + 1);
+          const uint32_t wv[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+#pragma unroll
+          for (int u = 0; u < 8; ++u) {
+            dst[2 * u] = bf16_lo(wv[u]);
+            dst[2 * u + 1] = bf16_hi(wv[u]);
+          }
           continue;
         }
         const int64_t row = seq * n + id;
@@ -184,7 +231,7 @@ __global__ void __launch_bounds__(kT) attn_simt_kernel(
 
 template <int HA, int DD>
 csa2_status run_simt(const void* q, const csa2_kv& kv, const int32_t* topk, int B, int Q, int k,
-                     float scale, void* out, float* lse, cudaStream_t stream) {
+                     float scale, void* out, float* lse, cudaStream_t stream, const AttnRows& rows) {
   const size_t smem = AttnSmem<HA, DD>::bytes;
   auto kern = kv.fmt == CSA2_KV_FP4 ? attn_simt_kernel<HA, DD, true> : attn_simt_kernel<HA, DD, false>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -194,32 +241,34 @@ csa2_status run_simt(const void* q, const csa2_kv& kv, const int32_t* topk, int 
   begin_launch(stream);
   kern<<<dim3(static_cast<unsigned>(Q), static_cast<unsigned>(B)), kT, smem, stream>>>(
       static_cast<const uint16_t*>(q), kv.data, kv.scales, kv.n, topk, k, scale,
-      static_cast<uint16_t*>(out), lse, device_error_word());
+      static_cast<uint16_t*>(out), lse, device_error_word(),
+      SimtRows{rows.n_visible, static_cast<const uint16_t*>(rows.win), rows.win_rows, rows.win_end,
+               rows.win ? rows.W : 0});
   note_launch(LK_ATTN, 1, stream);
   return check_launch("sparse_attn");
 }
 
 }  // namespace
 
-size_t sparse_attn_workspace(int B, int Q, int Ha, int D, int k, csa2_kv_fmt fmt) {
-  return sparse_attn_tc_workspace(B, Q, Ha, D, k, fmt);
+size_t sparse_attn_workspace(int B, int Q, int Ha, int D, int k, csa2_kv_fmt fmt, bool window) {
+  return sparse_attn_tc_workspace(B, Q, Ha, D, k, fmt, window);
 }
 
 csa2_status launch_sparse_attn(const void* q, const csa2_kv& kv, const int32_t* topk, int B,
                                int Q, int Ha, int k, float scale, void* out, float* lse, void* ws,
                                size_t ws_bytes, unsigned long long* sync_zeroed,
-                               cudaStream_t stream) {
+                               cudaStream_t stream, const AttnRows& rows) {
   if (B == 0 || Q == 0) return CSA2_OK;
   csa2_status s = launch_sparse_attn_tc(q, kv, topk, B, Q, Ha, k, scale, out, lse, ws, ws_bytes,
-                                        sync_zeroed, stream);
+                                        sync_zeroed, stream, rows);
   if (s != CSA2_ERR_UNSUPPORTED) return s;
   const int D = kv.dim;
-  if (Ha == 64 && D == 512) return run_simt<64, 512>(q, kv, topk, B, Q, k, scale, out, lse, stream);
-  if (Ha == 16 && D == 128) return run_simt<16, 128>(q, kv, topk, B, Q, k, scale, out, lse, stream);
-  if (Ha == 16 && D == 512) return run_simt<16, 512>(q, kv, topk, B, Q, k, scale, out, lse, stream);
-  if (Ha == 64 && D == 128) return run_simt<64, 128>(q, kv, topk, B, Q, k, scale, out, lse, stream);
-  if (Ha == 32 && D == 128) return run_simt<32, 128>(q, kv, topk, B, Q, k, scale, out, lse, stream);
-  if (Ha == 32 && D == 512) return run_simt<32, 512>(q, kv, topk, B, Q, k, scale, out, lse, stream);
+  if (Ha == 64 && D == 512) return run_simt<64, 512>(q, kv, topk, B, Q, k, scale, out, lse, stream, rows);
+  if (Ha == 16 && D == 128) return run_simt<16, 128>(q, kv, topk, B, Q, k, scale, out, lse, stream, rows);
+  if (Ha == 16 && D == 512) return run_simt<16, 512>(q, kv, topk, B, Q, k, scale, out, lse, stream, rows);
+  if (Ha == 64 && D == 128) return run_simt<64, 128>(q, kv, topk, B, Q, k, scale, out, lse, stream, rows);
+  if (Ha == 32 && D == 128) return run_simt<32, 128>(q, kv, topk, B, Q, k, scale, out, lse, stream, rows);
+  if (Ha == 32 && D == 512) return run_simt<32, 512>(q, kv, topk, B, Q, k, scale, out, lse, stream, rows);
   return fail(CSA2_ERR_UNSUPPORTED, "sparse_attn: (Ha=%d, D=%d) not instantiated", Ha, D);
 }
 

@@ -76,7 +76,13 @@ static_assert(kWeightsOff % 16 == 0 && kWeightsOff + 2 * kMaxTiles * HA * 4 <= k
 static_assert(SMEM_BYTES <= 232448, "shared memory");
 
 struct Params {
-  const int32_t* topk;             // [B*Q, k]
+  const int32_t* topk;             // [B*Q, k], or null: slot j is entry j (dense)
+  const int32_t* n_vis;            // dense: [B*Q] visible entries, or null (all k)
+  const uint16_t* win;             // window rows [B, win_rows, 512], or null (no window tile)
+  const int32_t* win_end;          // [B*Q] one past the query's last window row
+  int64_t win_rows;
+  int W;                           // window length
+  int T_sel;                       // tiles of selected rows; tile T_sel is the window tile
   const uint16_t* kv;              // [B, n, 512]
   uint16_t* out;                   // [B*Q, 64, 512]
   float* lse;                      // [B*Q, 64] or null
@@ -135,6 +141,34 @@ __device__ __forceinline__ unsigned ld_acquire_u32(const unsigned* p) {
   return v;
 }
 
+// Row of its source that row r of tile `tile` of query qi reads, or -1 for
+// an empty slot: a selected entry (tile < T_sel: the selection list, or the
+// slot itself when dense), or a window row (tile == T_sel).  An index
+// outside its source is recorded and treated as empty.
+__device__ __forceinline__ int tile_row(const Params& p, int64_t qi, int tile, int r) {
+  if (tile < p.T_sel) {
+    const int64_t pos = static_cast<int64_t>(tile) * kRows + r;
+    if (pos >= p.k) return -1;
+    if (!p.topk) {
+      const int64_t vis = p.n_vis ? p.n_vis[qi] : p.k;
+      return pos < vis ? static_cast<int>(pos) : -1;
+    }
+    const int id = p.topk[qi * p.k + pos];
+    if (id >= p.n || id < -1) {
+      raise_dev_error(p.err, DEVERR_BOUNDS);
+      return -1;
+    }
+    return id;
+  }
+  const int e = p.win_end[qi];
+  if (e < 0 || e > p.win_rows) {
+    raise_dev_error(p.err, DEVERR_BOUNDS);
+    return -1;
+  }
+  const int row = e - p.W + r;
+  return (r < p.W && row >= 0) ? row : -1;
+}
+
 // Drops a 128-byte line from L2 without writing it back (its content becomes
 // undefined); used on workspace lines that no one reads again.
 __device__ __forceinline__ void discard_l2_line(const void* p) {
@@ -182,12 +216,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   pdl_wait();                                  // the selection comes from the kernel before
   int32_t first_ids[8];
   if (warp >= 2 && n_waves > 0) {
-    const int32_t* ids = p.topk + static_cast<int64_t>(slot) * p.k;
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const int64_t pos = static_cast<int64_t>(tile) * kRows + grow0 + 16 * i;
-      first_ids[i] = pos < p.k ? ids[pos] : -1;
-    }
+    for (int i = 0; i < 8; ++i) first_ids[i] = tile_row(p, slot, tile, grow0 + 16 * i);
   }
 
   if (threadIdx.x == 0) {
@@ -285,24 +315,23 @@ __global__ void __launch_bounds__(kThreads, 1)
     // (grow0 + 16 i) & 7 == grow0 & 7: one swizzle per thread
     const uint32_t swz = static_cast<uint32_t>((c16 ^ (grow0 & 7)) << 4);
     auto issue_gather = [&](int64_t qi, const int32_t* pre) {   // pre: this wave's ids, or null
-      const uint16_t* base = p.kv + (qi / p.Q) * p.n * DV + c16 * 8;
-      const int32_t* ids = p.topk + qi * p.k;
+      const bool win_tile = tile >= p.T_sel;
+      const uint16_t* base = (win_tile ? p.win + (qi / p.Q) * p.win_rows * DV
+                                       : p.kv + (qi / p.Q) * p.n * DV) + c16 * 8;
       int64_t off[8];
+      uint32_t nbytes[8];
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
-        const int64_t pos = static_cast<int64_t>(tile) * kRows + grow0 + 16 * i;
-        int id = pre ? pre[i] : (pos < p.k ? ids[pos] : -1);
-        if (id >= p.n || id < -1) {
-          raise_dev_error(p.err, DEVERR_BOUNDS);
-          id = -1;
-        }
-        off[i] = static_cast<int64_t>(id >= 0 ? id : 0) * DV;     // empty slot: masked later
+        const int id = pre ? pre[i] : tile_row(p, qi, tile, grow0 + 16 * i);
+        off[i] = static_cast<int64_t>(id >= 0 ? id : 0) * DV;
+        nbytes[i] = id >= 0 ? 16u : 0u;            // empty slot: zero fill, nothing read
       }
 #pragma unroll 1
       for (int kb = 0; kb < kKB; ++kb) {          // not unrolled: one short body, re-executed
 #pragma unroll
         for (int i = 0; i < 8; ++i)
-          cp_async_16(sKV + kb * kKBBytes + (grow0 + 16 * i) * 128 + swz, base + off[i] + kb * 64, 16);
+          cp_async_16(sKV + kb * kKBBytes + (grow0 + 16 * i) * 128 + swz, base + off[i] + kb * 64,
+                      nbytes[i]);
         cp_async_commit();
       }
     };
@@ -324,9 +353,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int64_t w = 0; w < n_waves; ++w) {
       const int64_t qi = slot + w * p.G;
       const uint32_t par = static_cast<uint32_t>(w & 1);
-      const int64_t pos = static_cast<int64_t>(tile) * kRows + row;
-      const int64_t id = pos < p.k ? p.topk[qi * p.k + pos] : -1;
-      const bool valid = id >= 0 && id < p.n;
+      const bool valid = tile_row(p, qi, tile, row) >= 0;
       ok = ok && mbar_wait(s_full, par, abort_flag, p.err);
       float x[HA];
       if (ok) {
@@ -626,13 +653,15 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 struct Shape {
-  int T, dpc;
+  int T_sel, T, dpc;
 };
 
-Shape shape_for(int k) {
-  const int T = (k + kRows - 1) / kRows;
+// T_sel tiles of selected rows (k slots), plus one window tile when `win`.
+Shape shape_for(int k, bool win) {
+  const int T_sel = (k + kRows - 1) / kRows;
+  const int T = T_sel + (win ? 1 : 0);
   const int per = (DV + T - 1) / T;
-  return {T, (per + 3) / 4 * 4};
+  return {T_sel, T, (per + 3) / 4 * 4};
 }
 
 // CTAs of this kernel that fit on the device at once (cached), capped by the
@@ -674,28 +703,29 @@ WsLayout ws_layout(int64_t n_queries, Shape s) {
   return l;
 }
 
-bool applies(int Ha, int D, int k, csa2_kv_fmt fmt) {
-  if (fmt != CSA2_KV_BF16 || Ha != HA || D != DV || k <= 0) return false;
-  const Shape s = shape_for(k);
-  return s.T <= kMaxTiles && s.T <= kAttnMaxGrid;
+bool applies(int Ha, int D, int k, csa2_kv_fmt fmt, bool win) {
+  if (fmt != CSA2_KV_BF16 || Ha != HA || D != DV || k < 0) return false;
+  const Shape s = shape_for(k, win);
+  return s.T >= 1 && s.T <= kMaxTiles && s.T <= kAttnMaxGrid;
 }
 
 }  // namespace
 
-size_t sparse_attn_tc_workspace(int B, int Q, int Ha, int D, int k, csa2_kv_fmt fmt) {
-  if (!applies(Ha, D, k, fmt)) return 0;
-  return ws_layout(static_cast<int64_t>(B) * Q, shape_for(k)).total;
+size_t sparse_attn_tc_workspace(int B, int Q, int Ha, int D, int k, csa2_kv_fmt fmt, bool win) {
+  if (!applies(Ha, D, k, fmt, win)) return 0;
+  return ws_layout(static_cast<int64_t>(B) * Q, shape_for(k, win)).total;
 }
 
 csa2_status launch_sparse_attn_tc(const void* q, const csa2_kv& kv, const int32_t* topk, int B,
                                   int Q, int Ha, int k, float scale, void* out, float* lse,
                                   void* ws, size_t ws_bytes, unsigned long long* sync_zeroed,
-                                  cudaStream_t stream) {
+                                  cudaStream_t stream, const AttnRows& rows) {
   if (getenv("CSA2_ATTN_SIMT")) return CSA2_ERR_UNSUPPORTED;      // force the CUDA-core kernel
-  if (!applies(Ha, kv.dim, k, kv.fmt)) return CSA2_ERR_UNSUPPORTED;
+  const bool win = rows.win != nullptr;
+  if (!applies(Ha, kv.dim, k, kv.fmt, win)) return CSA2_ERR_UNSUPPORTED;
   const int64_t n_queries = static_cast<int64_t>(B) * Q;
   if (n_queries * HA > 0x7fffffffLL) return CSA2_ERR_UNSUPPORTED;
-  const Shape s = shape_for(k);
+  const Shape s = shape_for(k, win);
   const int cap = resident_ctas();
   if (cap < s.T) return CSA2_ERR_UNSUPPORTED;
   const WsLayout lay = ws_layout(n_queries, s);
@@ -706,6 +736,12 @@ csa2_status launch_sparse_attn_tc(const void* q, const csa2_kv& kv, const int32_
   CSA2_TRY(make_tensor_map_bf16_2d(&qmap, q, static_cast<uint64_t>(n_queries) * HA, DV, DV * 2, 64, HA));
   Params p;
   p.topk = topk;
+  p.n_vis = rows.n_visible;
+  p.win = static_cast<const uint16_t*>(rows.win);
+  p.win_end = rows.win_end;
+  p.win_rows = rows.win_rows;
+  p.W = rows.W;
+  p.T_sel = s.T_sel;
   p.kv = static_cast<const uint16_t*>(kv.data);
   p.out = static_cast<uint16_t*>(out);
   p.lse = lse;

@@ -75,7 +75,73 @@ __global__ void __launch_bounds__(256) compress_kernel(
                             static_cast<int64_t>(j) * D + ch0) = o;
 }
 
+// HCA compression ("读完这篇，你就搞懂 DeepSeek v4 了", HCA 压缩机制, eq. 10 and
+// 11): entry j is the per-channel softmax-weighted sum of the m tokens of
+// block j alone (no overlap with the block before), bias [m, D] indexed by the
+// position in the block.  Blocks are long (m up to 1024), so each thread runs
+// one pass over its block with a running max (the sums are rescaled when the
+// max grows) instead of the two passes of the overlapping kernel.
+__global__ void __launch_bounds__(256) compress_hca_kernel(
+    const uint16_t* __restrict__ c, const float* __restrict__ z, const float* __restrict__ bias,
+    int N, int D, int m, int64_t t_in, uint16_t* __restrict__ out, int64_t out_bstride) {
+  const int groups = D / 8;
+  const int64_t gid = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x;
+  const int b = blockIdx.y;
+  if (gid >= static_cast<int64_t>(N) * groups) return;
+  const int j = static_cast<int>(gid / groups);
+  const int ch0 = static_cast<int>(gid % groups) * 8;
+  const int64_t seq = static_cast<int64_t>(b) * t_in * D;
+  const int64_t first = static_cast<int64_t>(j) * m;
+
+  float mx[8], den[8], num[8];
+#pragma unroll
+  for (int u = 0; u < 8; ++u) { mx[u] = -INFINITY; den[u] = 0.0f; num[u] = 0.0f; }
+  for (int w = 0; w < m; ++w) {
+    float zz[8], bb[8];
+    load8f(z + seq + (first + w) * D + ch0, zz);
+    load8f(bias + static_cast<int64_t>(w) * D + ch0, bb);
+    const uint4 cv = __ldg(reinterpret_cast<const uint4*>(c + seq + (first + w) * D + ch0));
+    const float cc[8] = {bf16_lo(cv.x), bf16_hi(cv.x), bf16_lo(cv.y), bf16_hi(cv.y),
+                         bf16_lo(cv.z), bf16_hi(cv.z), bf16_lo(cv.w), bf16_hi(cv.w)};
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const float x = zz[u] + bb[u];
+      if (x > mx[u]) {                       // a new max: rescale what is summed so far
+        const float s = expf(mx[u] - x);     // 0 while nothing is summed (mx = -inf)
+        den[u] *= s;
+        num[u] *= s;
+        mx[u] = x;
+      }
+      const float p = x == -INFINITY ? 0.0f : expf(x - mx[u]);
+      den[u] += p;
+      num[u] = fmaf(p, cc[u], num[u]);
+    }
+  }
+  uint4 o;
+  o.x = pack_bf16x2(num[0] / den[0], num[1] / den[1]);
+  o.y = pack_bf16x2(num[2] / den[2], num[3] / den[3]);
+  o.z = pack_bf16x2(num[4] / den[4], num[5] / den[5]);
+  o.w = pack_bf16x2(num[6] / den[6], num[7] / den[7]);
+  *reinterpret_cast<uint4*>(out + static_cast<int64_t>(b) * out_bstride +
+                            static_cast<int64_t>(j) * D + ch0) = o;
+}
+
 }  // namespace
+
+csa2_status launch_compress_hca(const void* c, const float* z, const float* bias, int B, int64_t T,
+                                int D, int m, void* out, int64_t out_bstride, cudaStream_t stream) {
+  const int64_t N = T / m;
+  if (N == 0 || B == 0) return CSA2_OK;
+  const int64_t work = N * (D / 8);
+  const int threads = 256;
+  dim3 grid(static_cast<unsigned>((work + threads - 1) / threads), static_cast<unsigned>(B));
+  begin_launch(stream);
+  compress_hca_kernel<<<grid, threads, 0, stream>>>(static_cast<const uint16_t*>(c), z, bias,
+                                                    static_cast<int>(N), D, m, T,
+                                                    static_cast<uint16_t*>(out), out_bstride);
+  note_launch(LK_COMPRESS, 1, stream);
+  return check_launch("compress_hca");
+}
 
 csa2_status launch_compress(const void* c, const float* z, const float* bias, int B, int64_t T,
                             int D, int m, int halo, void* out, int64_t out_bstride,

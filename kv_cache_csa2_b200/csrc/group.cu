@@ -29,7 +29,10 @@ struct csa2_group {
   int32_t* pool = nullptr;   // [B, Q, P]   pool of the last Full layer (P > 0)
   void* ws = nullptr;        // scores + selection state, then attention workspace
   size_t ws_bytes = 0;
-  unsigned long long* attn_sync = nullptr;  // attention arrival counters, zeroed once
+  // attention arrival counters, zeroed once: [0, kAttnMaxGrid) for layers
+  // without a window branch, [kAttnMaxGrid, 2 kAttnMaxGrid) for layers with
+  // one (each launch shape keeps its own counters consistent)
+  unsigned long long* attn_sync = nullptr;
   bool have_full = false;
   csa2_kv kv{};              // registered by the last Full layer (not owned)
   const void* index_k = nullptr;
@@ -65,14 +68,16 @@ csa2_status csa2_group_create(csa2_group** group, const csa2_group_desc* d) {
     const size_t w2 = csa2_index_topk_workspace(d->B, d->Q, d->N, d->P, d->k, 0);
     if (w2 > ws) ws = w2;
   }
-  const size_t wa = csa2_sparse_attn_workspace(d->B, d->Q, d->Ha, d->D, d->k, d->kv_fmt);
+  size_t wa = csa2_sparse_attn_workspace(d->B, d->Q, d->Ha, d->D, d->k, d->kv_fmt);
+  const size_t wa2 = csa2_sparse_attn_swa_workspace(d->B, d->Q, d->Ha, d->D, d->k, d->kv_fmt);
+  if (wa2 > wa) wa = wa2;
   if (wa > ws) ws = wa;
   g->ws_bytes = a256(ws);
   cudaError_t e = cudaMalloc(&g->topk, a256(rows * d->k * sizeof(int32_t)));
   if (e == cudaSuccess && d->P > 0) e = cudaMalloc(&g->pool, a256(rows * d->P * sizeof(int32_t)));
   if (e == cudaSuccess) e = cudaMalloc(&g->ws, g->ws_bytes);
-  if (e == cudaSuccess) e = cudaMalloc(&g->attn_sync, kAttnMaxGrid * sizeof(unsigned long long));
-  if (e == cudaSuccess) e = cudaMemset(g->attn_sync, 0, kAttnMaxGrid * sizeof(unsigned long long));
+  if (e == cudaSuccess) e = cudaMalloc(&g->attn_sync, 2 * kAttnMaxGrid * sizeof(unsigned long long));
+  if (e == cudaSuccess) e = cudaMemset(g->attn_sync, 0, 2 * kAttnMaxGrid * sizeof(unsigned long long));
   if (e != cudaSuccess) {
     cudaGetLastError();
     csa2_group_destroy(g);
@@ -153,9 +158,17 @@ csa2_status csa2_group_layer(csa2_group* g, int layer, const csa2_layer_io* io,
                         d.P, d.k, g->topk, nullptr, 0, d.act, g->ws, g->ws_bytes, stream);
     if (s != CSA2_OK) return s;
   }
+  AttnRows rows;
+  if (io->swa_kv) {             // this layer's own sliding-window branch
+    rows.win = io->swa_kv;
+    rows.win_rows = io->swa_rows;
+    rows.win_end = io->swa_end;
+    rows.W = io->swa_window;
+  }
   return sparse_attn_checked(mode, io->q_attn, &g->kv, g->topk, d.B, d.Q, d.Ha, d.k, d.scale,
-                             io->out, io->lse, g->ws, g->ws_bytes, g->attn_sync,
-                             reinterpret_cast<cudaStream_t>(stream));
+                             io->out, io->lse, g->ws, g->ws_bytes,
+                             g->attn_sync + (io->swa_kv ? kAttnMaxGrid : 0),
+                             reinterpret_cast<cudaStream_t>(stream), rows);
 }
 
 }  // extern "C"

@@ -10,6 +10,10 @@ namespace csa2 {
 csa2_status launch_compress(const void* c, const float* z, const float* bias, int B, int64_t T,
                             int D, int m, int halo, void* out, int64_t out_bstride,
                             cudaStream_t stream);
+// HCA compression: entry j is the softmax-weighted sum of block j alone.
+constexpr int kMaxHcaBlock = 1024;
+csa2_status launch_compress_hca(const void* c, const float* z, const float* bias, int B, int64_t T,
+                                int D, int m, void* out, int64_t out_bstride, cudaStream_t stream);
 
 // Words of device memory that the scoring kernel clears at its start for the
 // selection launched after it, so that no separate memset sits between the
@@ -64,19 +68,36 @@ csa2_status launch_select_topk(const float* scores, int64_t rows, int64_t L, int
 // CTAs that fit at once); sizes its workspace and its arrival counters.
 constexpr int kAttnMaxGrid = 160;
 
-size_t sparse_attn_workspace(int B, int Q, int Ha, int D, int k, csa2_kv_fmt fmt);
+// Rows an attention launch takes besides a selection list.
+//  - topk == NULL (dense): slot j of a query is entry j, visible while
+//    j < n_visible[query] (all k = kv.n slots when n_visible is NULL).
+//  - win != NULL: one more tile of rows per query, from a sliding window of
+//    uncompressed rows (bf16 [B, win_rows, D]): query qi takes rows
+//    [max(0, e - W), e) with e = win_end[qi] (0 <= e <= win_rows), in the same
+//    softmax as its other rows.
+struct AttnRows {
+  const int32_t* n_visible = nullptr;
+  const void* win = nullptr;
+  int64_t win_rows = 0;
+  const int32_t* win_end = nullptr;
+  int W = 0;
+};
+constexpr int kMaxWindow = 128;
+
+size_t sparse_attn_workspace(int B, int Q, int Ha, int D, int k, csa2_kv_fmt fmt, bool window = false);
 // sync_zeroed: kAttnMaxGrid * 8 bytes of per-CTA flags that were zero before
 // their first use and are left consistent by every launch (a layer group's),
 // or NULL to take them from the workspace and clear them on the stream.
 csa2_status launch_sparse_attn(const void* q, const csa2_kv& kv, const int32_t* topk, int B,
                                int Q, int Ha, int k, float scale, void* out, float* lse, void* ws,
                                size_t ws_bytes, unsigned long long* sync_zeroed,
-                               cudaStream_t stream);
+                               cudaStream_t stream, const AttnRows& rows = AttnRows());
 // csa2_sparse_attn's argument checks, then launch_sparse_attn.
 csa2_status sparse_attn_checked(csa2_mode mode, const void* q, const csa2_kv* kv,
                                 const int32_t* topk, int B, int Q, int Ha, int k, float scale,
                                 void* out, float* lse, void* workspace, size_t workspace_bytes,
-                                unsigned long long* sync_zeroed, cudaStream_t stream);
+                                unsigned long long* sync_zeroed, cudaStream_t stream,
+                                const AttnRows& rows = AttnRows());
 
 csa2_status launch_fp4_pack(const void* x, int64_t rows, int D, uint8_t* codes, uint8_t* scales,
                             cudaStream_t stream);
