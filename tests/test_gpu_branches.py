@@ -109,7 +109,7 @@ def _swa_case(r, B, Q, Ha, D, N, k, R, W, prefill):
     (64, 512, 5000, 2048, 128, 128, False, False),     # decode, tensor-core kernel, 17 tiles
     (64, 512, 3000, 300, 200, 128, True, False),       # prefill-like window ends
     (64, 512, 900, 0, 64, 64, True, False),            # no selected entries: the window alone
-    (64, 512, 4000, 4096, 128, 100, False, False),     # W < 128
+    (64, 512, 5000, 4096, 128, 100, False, False),     # W < 128, 33 tiles (two waves)
     (16, 128, 3000, 256, 160, 128, True, True),        # CUDA-core kernel, FP4 main KV, bf16 window
     (16, 128, 500, 33, 100, 64, False, False),
 ])
