@@ -264,6 +264,26 @@ def sparse_attn(q: np.ndarray, kv: np.ndarray, topk: np.ndarray, scale: float):
     return o, round_to_bf16(o), lse
 
 
+def index_scores_fp4(q: np.ndarray, w: np.ndarray, k: np.ndarray,
+                     n_visible: np.ndarray | None = None,
+                     pool: np.ndarray | None = None,
+                     act: str = "relu") -> np.ndarray:
+    """The lightning indexer with FP4 queries and keys and BF16 scores (V4
+    explainer, FP4量化感知训练: the indexer's q and K are stored in FP4 while the
+    scores are kept in BF16).  Readings: q and K use the main-KV FP4 format of
+    "Recall之王" (E2M1 values, one E4M3 scale per 16 channels along d, fp4_pack);
+    the score is eq. 8 over the dequantised values, computed exactly and
+    rounded once to bf16 (unscored slots stay -inf).
+
+    q: [B, Q, H, d], k: [B, N, d] values before quantisation (d % 16 == 0).
+    Returns float64 [B, Q, N or P] holding bf16 values."""
+    q = np.asarray(q, dtype=np.float64)
+    k = np.asarray(k, dtype=np.float64)
+    qd = fp4_unpack(*fp4_pack(q.reshape(-1, q.shape[-1]))).reshape(q.shape)
+    kd = fp4_unpack(*fp4_pack(k.reshape(-1, k.shape[-1]))).reshape(k.shape)
+    return round_to_bf16(index_scores(qd, w, kd, n_visible=n_visible, pool=pool, act=act))
+
+
 # ----------------------------------------------------------------------------
 # sliding-window branch and its merge with the CSA2 branch
 # ----------------------------------------------------------------------------

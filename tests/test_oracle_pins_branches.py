@@ -180,3 +180,59 @@ def test_group_layer_with_window_merges_its_branch():
         o, _, lse = (O.sparse_attn_swa(layers[i]["q_attn"], kv, res[i]["topk"], win, we, W, 0.3) if i == 0
                      else O.sparse_attn(layers[i]["q_attn"], kv, res[i]["topk"], 0.3))
         assert np.array_equal(res[i]["o"], o) and np.array_equal(res[i]["lse"], lse)
+
+
+# ------------------------------------------------------------------ FP4 indexer, bf16 scores
+
+def _fp4_exact_rows(r, shape, scale_exp):
+    """Rows whose every 16-channel block holds E2M1 values times one power-of-two
+    scale, with a +-6 in each block (so quantising them again changes nothing)."""
+    grid = np.array([0, 0.5, 1, 1.5, 2, 3, 4, 6])
+    v = grid[r.integers(0, 8, shape)] * np.where(r.random(shape) < 0.5, -1.0, 1.0)
+    v.reshape(-1, 16)[:, 0] = 6.0
+    return v * 2.0 ** scale_exp
+
+
+def test_index_fp4_golden():
+    """d = 16, one head: q = (6, 1.5, 0, ..), k = (1.5, 1, 0, ..), both FP4
+    exact with scale 1 (absmax 6); q.k = 9 + 1.5 = 10.5; w = 0.1 gives
+    1.05000001...; bfloat16 keeps 8 significant bits, so in [1, 2) its values
+    are 1/128 apart and the neighbours are 1 + 6/128 = 1.046875 (0.0031 away)
+    and 1 + 7/128 = 1.0546875 (0.0047 away): the score is 1.046875."""
+    q = np.zeros((1, 1, 1, 16))
+    q[..., 0], q[..., 1] = 6.0, 1.5
+    k = np.zeros((1, 2, 16))
+    k[0, 0, 0], k[0, 0, 1], k[0, 0, 2] = 1.5, 1.0, 6.0        # the 6 pairs with q's 0
+    k[0, 1, 0] = -6.0                                         # q.k = -36: ReLU gives 0
+    w = np.array([[[np.float32(0.1)]]], dtype=np.float64)
+    s = O.index_scores_fp4(q, w, k)
+    assert s[0, 0, 0] == 1.046875 and s[0, 0, 1] == 0.0
+
+
+def test_index_fp4_on_fp4_exact_inputs_is_rounded_exact_score():
+    r = np.random.default_rng(46)
+    q = _fp4_exact_rows(r, (2, 3, 4, 64), -3)
+    k = _fp4_exact_rows(r, (2, 50, 64), -2)
+    w = r.random((2, 3, 4))
+    nv = np.array([[50, 10, 0], [1, 49, 50]])
+    s = O.index_scores_fp4(q, w, k, n_visible=nv)
+    assert np.array_equal(s, O.round_to_bf16(O.index_scores(q, w, k, n_visible=nv)))
+    assert np.array_equal(s, O.round_to_bf16(s))              # bf16 values
+    assert np.all(np.isneginf(s[0, 2])) and np.all(np.isneginf(s[1, 0, 1:]))
+
+
+def test_index_fp4_quantises_q_and_k_like_the_main_kv_format():
+    r = np.random.default_rng(47)
+    q = r.standard_normal((1, 2, 3, 32))
+    k = r.standard_normal((1, 40, 32))
+    w = r.random((1, 2, 3))
+    qd = O.fp4_unpack(*O.fp4_pack(q.reshape(-1, 32))).reshape(q.shape)
+    kd = O.fp4_unpack(*O.fp4_pack(k.reshape(-1, 32))).reshape(k.shape)
+    s = O.index_scores_fp4(q, w, k)
+    # scores over the dequantised values, computed directly (ReLU, weighted head sum)
+    direct = np.einsum("bqh,bqhn->bqn", w, np.maximum(np.einsum("bqhd,bnd->bqhn", qd, kd), 0.0))
+    assert np.allclose(s, direct, rtol=2.0 ** -8, atol=0)
+    assert not np.allclose(s, O.index_scores(q, w, k), rtol=1e-3)   # quantisation matters
+    pool = np.sort(r.choice(40, (1, 2, 7)), axis=-1)
+    sp = O.index_scores_fp4(q, w, k, pool=pool)
+    assert np.array_equal(sp, np.take_along_axis(s, pool, axis=-1))
