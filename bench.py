@@ -213,6 +213,7 @@ def algorithmic_bytes(wl):
     if wl.P and n_re:
         out["index_pool"] = (n_re * (rows * wl.P * (wl.d * 2 + 4) + qidx), n_re)
     attn = wl.n_layers * (rows * wl.k * (kv_row + 4) + rows * wl.Ha * (wl.D * 2 * 2 + 4))
+    attn += wl.n_layers * wl.B * wl.swa * wl.D * 2          # each layer's window rows
     out["attn"] = (attn, wl.n_layers)
     if wl.compress_new_tokens:        # raw tokens c (bf16) and z (f32) in, entries (bf16) out
         t_in = wl.compress_new_tokens + (wl.m if wl.halo else 0)
@@ -237,7 +238,7 @@ def algorithmic_flops(wl):
     out = {"index_scores": per * visible * (n_full + (n_re if wl.P == 0 else 0))}
     if wl.P and n_re:
         out["index_pool"] = per * rows * wl.P * n_re
-    out["attn"] = wl.n_layers * rows * wl.k * wl.Ha * wl.D * 4
+    out["attn"] = wl.n_layers * rows * (wl.k + wl.swa) * wl.Ha * wl.D * 4
     return out
 
 
@@ -269,6 +270,8 @@ def device_inputs(wl, inp, torch, device):
          "layers": []}
     for L in inp["layers"]:
         e = {"q_attn": bf(L["q_attn"])}
+        if "win" in L:
+            e["swa"] = (bf(L["win"]), torch.from_numpy(L["win_end"]).to(device), wl.swa)
         if "q_index" in L:
             e["q_index"] = bf(L["q_index"])
             e["w_index"] = torch.from_numpy(L["w_index"]).to(device)
@@ -328,7 +331,7 @@ def run_ours(args, wl, world, rank, local):
     def layer(i):
         if i == 0 and compress is not None:
             compress()
-        g.layer(i, D["layers"][i]["q_attn"], outs[i], lses[i], **kws[i])
+        g.layer(i, D["layers"][i]["q_attn"], outs[i], lses[i], swa=D["layers"][i].get("swa"), **kws[i])
 
     flush_buf = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device=dev)
 
@@ -520,7 +523,7 @@ def run_ours(args, wl, world, rank, local):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 4),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic (seeded N(0,1)/U(0,1) inputs of the workload's shapes)",
-        "config": {"workload": wl.name, "B": wl.B, "Q": wl.Q, "L": wl.L, "m": wl.m, "N": wl.N,
+        "config": {"workload": wl.name, "B": wl.B, "Q": wl.Q, "L": wl.L, "m": wl.m, "N": wl.N, "swa": wl.swa,
                    "D": wl.D, "Ha": wl.Ha, "Hi": wl.Hi, "d": wl.d, "k": wl.k, "P": wl.P,
                    "modes": ",".join(wl.modes), "kv": "fp4" if wl.kv_fp4 else "bf16",
                    "l2": "flushed before every layer (2x L2 write outside the layer's events); "
@@ -588,6 +591,8 @@ def oracle_queries(wl, inp, queries):
         layers = []
         for L in inp["layers"]:
             d = {"q_attn": O.bf16_bits_to_float(L["q_attn"][b:b + 1, t:t + 1])}
+            if "win" in L:
+                d["swa"] = (O.bf16_bits_to_float(L["win"][b:b + 1]), L["win_end"][b:b + 1, t:t + 1], wl.swa)
             if "q_index" in L:
                 d["q_index"] = O.bf16_bits_to_float(L["q_index"][b:b + 1, t:t + 1])
                 d["w_index"] = L["w_index"][b:b + 1, t:t + 1].astype(np.float64)
@@ -658,41 +663,126 @@ def run_reference(args, wl, world, rank):
 
 # ---------------------------------------------------------------------------- kernel cases
 
-def run_kernel_case(name, reps=4):
-    """One library call of the c4 group on seeded synthetic inputs, `reps` times
-    (a short program for ncu captures of one kernel; prints one JSON line).
-      attn     csa2_sparse_attn, 8 queries x 64 heads x 512, k = 2048, 32768
-               entries per sequence (the kernel gathers 2048 rows either way)
-      full     csa2_index_topk(FULL) over 8 x 262144 entries, pool 16384 + top 2048
-      reindex  csa2_index_topk(REINDEX) inside a 16384-slot pool, top 2048"""
+KERNEL_CASES = ("attn", "full", "reindex", "attn_swa", "dense", "compress_hca", "full_fp4",
+                "reindex_fp4", "fused_prefill")
+
+
+def run_kernel_case(name, reps=4, timed=False):
+    """One library call on seeded synthetic inputs of one workload's shapes,
+    `reps` times (the short program the ncu captures use; prints one JSON
+    line).  With `timed`, each call runs after an L2 flush, bracketed by CUDA
+    events on the launching stream, and the line carries the median time and
+    the algorithmic bytes and flops of one call with their roofline fraction.
+      attn           csa2_sparse_attn, 8 queries x 64 heads x 512, k = 2048
+      full           csa2_index_topk(FULL) over 8 x 262144 entries, pool 16384 + top 2048
+      reindex        csa2_index_topk(REINDEX) inside a 16384-slot pool, top 2048
+      attn_swa       attn plus each query's 128-row sliding window (csa2_sparse_attn_swa)
+      dense          HCA attention: 8 queries over 8192 entries (1M tokens / 128)
+      compress_hca   HCA compression of 8 x 8192 tokens into groups of 128 (D = 512)
+      full_fp4       full with the FP4 indexer (FP4 q and K, bf16 scores)
+      reindex_fp4    reindex with the FP4 indexer
+      fused_prefill  csa2_index_topk(FULL) of a 4096-query prefill chunk over 262144
+                     entries, top 2048: the fused indexer + streaming top-k"""
     import torch
     import kv_cache_csa2_b200 as K
     g = torch.Generator(device="cuda").manual_seed(0)
-    B = 8
-    if name == "attn":
-        N, D, Ha, k = 32768, 512, 64, 2048
-        kv = torch.randn(B, N, D, device="cuda", generator=g).to(torch.bfloat16)
-        q = torch.randn(B, 1, Ha, D, device="cuda", generator=g).to(torch.bfloat16)
-        ids = torch.stack([torch.sort(torch.randperm(N, device="cuda", generator=g)[:k])[0] for _ in range(B)])
-        topk = ids.view(B, 1, k).to(torch.int32)
-        for _ in range(reps):
-            K.csa2_sparse_attn(q, kv, topk, D ** -0.5)
-    else:
-        N = 262144
-        q = (torch.randn(B, 1, 64, 128, device="cuda", generator=g) / 11.3).to(torch.bfloat16)
-        w = torch.rand(B, 1, 64, device="cuda", generator=g)
-        k = (torch.randn(B, N, 128, device="cuda", generator=g) / 11.3).to(torch.bfloat16)
-        if name == "full":
-            for _ in range(reps):
-                K.csa2_index_topk(K.FULL, q, w, k, 2048, pool_size=16384)
+    B, D, Ha, k_sel = 8, 512, 64, 2048
+    flops, nbytes = 0.0, 0.0
+
+    def randn(*shape, std=1.0):
+        return (torch.randn(*shape, device="cuda", generator=g) * std).to(torch.bfloat16)
+
+    def sel_ids(N, k):
+        return torch.stack([torch.sort(torch.randperm(N, device="cuda", generator=g)[:k])[0]
+                            for _ in range(B)]).view(B, 1, k).to(torch.int32)
+
+    if name in ("attn", "attn_swa"):
+        N = 32768
+        kv, q, topk = randn(B, N, D), randn(B, 1, Ha, D), sel_ids(N, k_sel)
+        nbytes = B * k_sel * (D * 2 + 4) + B * Ha * (D * 4 + 4)
+        flops = 4.0 * B * k_sel * Ha * D
+        if name == "attn":
+            call = lambda: K.csa2_sparse_attn(q, kv, topk, D ** -0.5)  # noqa: E731
         else:
-            ids = torch.stack([torch.sort(torch.randperm(N, device="cuda", generator=g)[:16384])[0] for _ in range(B)])
-            pool = ids.view(B, 1, 16384).to(torch.int32)
-            for _ in range(reps):
-                K.csa2_index_topk(K.REINDEX, q, w, k, 2048, pool_in=pool)
-    torch.cuda.synchronize()
+            win = randn(B, 128, D)
+            we = torch.full((B, 1), 128, dtype=torch.int32, device="cuda")
+            nbytes += B * 128 * D * 2
+            flops += 4.0 * B * 128 * Ha * D
+            call = lambda: K.csa2_sparse_attn_swa(q, kv, topk, D ** -0.5, win, we, 128)  # noqa: E731
+    elif name == "dense":
+        N = 8192
+        kv, q = randn(B, N, D), randn(B, 1, Ha, D)
+        nbytes = B * N * D * 2 + B * Ha * (D * 4 + 4)
+        flops = 4.0 * B * N * Ha * D
+        call = lambda: K.csa2_dense_attn(q, kv, D ** -0.5)  # noqa: E731
+    elif name == "compress_hca":
+        T, m = 8192, 128
+        c = randn(B, T, D)
+        z = torch.randn(B, T, D, device="cuda", generator=g)
+        bias = torch.randn(m, D, device="cuda", generator=g)
+        nbytes = B * T * D * 6 + B * (T // m) * D * 2 + m * D * 4
+        call = lambda: K.csa2_compress_hca(c, z, bias, m)  # noqa: E731
+    elif name == "fused_prefill":
+        Q, N = 4096, 262144
+        q = randn(1, Q, 64, 128)
+        w = torch.randn(1, Q, 64, device="cuda", generator=g)
+        kk = randn(1, N, 128)
+        nv = torch.arange(N - Q + 1, N + 1, dtype=torch.int32, device="cuda").view(1, Q)
+        flops = 2.0 * 64 * 128 * float(nv.sum().item())
+        nbytes = N * 128 * 2 + Q * 64 * (128 * 2 + 4) + Q * k_sel * 4
+        call = lambda: K.csa2_index_topk(K.FULL, q, w, kk, k_sel, n_visible=nv)  # noqa: E731
+    else:
+        N, P = 262144, 16384
+        fp4 = name.endswith("_fp4")
+        q = randn(B, 1, 64, 128, std=1 / 11.3)
+        w = torch.rand(B, 1, 64, device="cuda", generator=g)
+        kk = randn(B, N, 128, std=1 / 11.3)
+        row = 128 // 2 + 128 // 16 if fp4 else 128 * 2
+        pool = sel_ids(N, P) if name.startswith("reindex") else None
+        scored = B * (P if pool is not None else N)
+        nbytes = scored * (row + (4 if pool is not None else 0)) + B * k_sel * 4 + (B * P * 4 if pool is None else 0)
+        flops = 2.0 * scored * 64 * 128
+        if fp4:
+            qc, qs = K.csa2_fp4_pack(q)
+            kc, ks = K.csa2_fp4_pack(kk)
+            if pool is None:
+                call = lambda: K.csa2_index_topk_fp4(K.FULL, qc, qs, w, kc, ks, k_sel, pool_size=P)  # noqa: E731
+            else:
+                call = lambda: K.csa2_index_topk_fp4(K.REINDEX, qc, qs, w, kc, ks, k_sel, pool_in=pool)  # noqa: E731
+        elif pool is None:
+            call = lambda: K.csa2_index_topk(K.FULL, q, w, kk, k_sel, pool_size=P)  # noqa: E731
+        else:
+            call = lambda: K.csa2_index_topk(K.REINDEX, q, w, kk, k_sel, pool_in=pool)  # noqa: E731
+    res = {"kernel_case": name, "reps": reps, "ok": True}
+    if not timed:
+        for _ in range(reps):
+            call()
+        torch.cuda.synchronize()
+        K.csa2_device_error()
+        return res
+    flush_buf = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device="cuda")
+    for _ in range(3):
+        flush_buf.fill_(1.0)
+        call()
+    times = []
+    for _ in range(reps):
+        flush_buf.fill_(1.0)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        call()
+        e1.record()
+        e1.synchronize()
+        times.append(e0.elapsed_time(e1))
     K.csa2_device_error()
-    return {"kernel_case": name, "reps": reps, "ok": True}
+    t = statistics.median(times) / 1e3
+    hbm, _ = measured_hbm_gbs()
+    tflops, tsrc = measured_tflops(t)
+    res.update(us=round(t * 1e6, 2), algorithmic_bytes=int(nbytes), algorithmic_flops=int(flops),
+               achieved_gbs=round(nbytes / t / 1e9, 1), achieved_tflops=round(flops / t / 1e12, 2),
+               hbm_frac=round(nbytes / t / 1e9 / hbm, 4), tensor_frac=round(flops / t / 1e12 / tflops, 4),
+               tensor_peak=tflops, tensor_peak_source=tsrc,
+               l2="flushed before every call (2x L2 write outside the events)")
+    return res
 
 
 # ---------------------------------------------------------------------------- main
@@ -702,17 +792,21 @@ def main(argv=None):
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--config", type=int, default=4, choices=[1, 2, 3, 4, 5])
+    ap.add_argument("--config", type=int, default=4, choices=[1, 2, 3, 4, 5, 6])
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--cpu-budget", type=float, default=20.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--eager", action="store_true", help="launch layers eagerly instead of CUDA graphs")
-    ap.add_argument("--kernel-case", choices=["attn", "full", "reindex"],
-                    help="run one library call of the group 4 times and exit (for ncu captures)")
+    ap.add_argument("--kernel-case", choices=KERNEL_CASES,
+                    help="run one library call of a workload 4 times and exit (for ncu captures)")
+    ap.add_argument("--timed", action="store_true",
+                    help="with --kernel-case: time --steps calls (L2 flushed before each) and report "
+                         "the median with its roofline fraction")
     args = ap.parse_args(argv)
     if args.kernel_case:
-        print(json.dumps(run_kernel_case(args.kernel_case)), flush=True)
+        reps = args.steps if args.timed else 4
+        print(json.dumps(run_kernel_case(args.kernel_case, reps=reps, timed=args.timed)), flush=True)
         return
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

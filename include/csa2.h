@@ -196,6 +196,34 @@ csa2_status csa2_index_topk(csa2_mode mode, const void* q, const float* w, const
                             int32_t* pool_out, int P_out, csa2_index_act act, void* workspace,
                             size_t workspace_bytes, csa2_stream stream);
 
+/* (a2 + a3, FP4 variant) The lightning indexer with FP4 queries and keys and
+ * BF16 scores.  [V4] FP4量化感知训练: the indexer's q and K are kept in FP4,
+ * its scores in BF16.  q and K use the FP4 format of csa2_fp4_pack (E2M1
+ * codes, channel 2i in the low nibble, one E4M3 scale per 16 channels along
+ * d).  Each score is eq. (8) over the dequantised values (exact products, f32
+ * accumulation) rounded once to bf16 (nearest even); unscored slots are -inf.
+ *   q_codes uint8 [B, Q, H, d/2]   q_scales uint8 [B, Q, H, d/16]   w f32 [B, Q, H]
+ *   k_codes uint8 [B, N, d/2]      k_scales uint8 [B, N, d/16]
+ *   n_visible, pool, P, act: as csa2_index_scores
+ *   scores  bf16 [B, Q, N] (no pool) or [B, Q, P]
+ * Requires d in {64, 128}, H <= 64; k_codes 16-byte aligned, q_codes 8-byte
+ * aligned, k_scales d/16-byte aligned.  Pool entries outside [0, N) other
+ * than -1 are recorded as CSA2_ERR_BOUNDS and scored -inf. */
+csa2_status csa2_index_scores_fp4(const uint8_t* q_codes, const uint8_t* q_scales, const float* w,
+                                  const uint8_t* k_codes, const uint8_t* k_scales, int B, int Q,
+                                  int H, int d, int64_t N, const int32_t* n_visible,
+                                  const int32_t* pool, int P, csa2_index_act act, void* scores,
+                                  csa2_stream stream);
+/* csa2_index_topk with the FP4 indexer: the same modes, outputs, order and
+ * errors, the selection taken over the bf16 scores (ties to the lower
+ * position).  workspace: csa2_index_topk_workspace(...) bytes. */
+csa2_status csa2_index_topk_fp4(csa2_mode mode, const uint8_t* q_codes, const uint8_t* q_scales,
+                                const float* w, const uint8_t* k_codes, const uint8_t* k_scales,
+                                int B, int Q, int H, int d, int64_t N, const int32_t* n_visible,
+                                const int32_t* pool_in, int P_in, int k_top, int32_t* topk_out,
+                                int32_t* pool_out, int P_out, csa2_index_act act, void* workspace,
+                                size_t workspace_bytes, csa2_stream stream);
+
 /* ------------------------------------------------------------------------ */
 /* (a4) Shared-KV sparse attention.  [V4] 注意力计算, eq. (9): every query head
  * attends, with softmax(scale * q_h . e_j), over the selected entries e_j,

@@ -15,6 +15,7 @@ __all__ = [
     "ACT_IDENTITY", "csa2_compress", "csa2_index_scores", "csa2_select_topk", "csa2_select_topk_noalloc",
     "csa2_index_topk",
     "csa2_sparse_attn", "csa2_sparse_attn_swa", "csa2_dense_attn", "csa2_compress_hca",
+    "csa2_index_scores_fp4", "csa2_index_topk_fp4",
     "csa2_fp4_pack", "csa2_fp4_unpack", "Group", "csa2_device_error",
     "launch_counts", "reset_launch_counts", "set_fault", "set_device_wait", "EXPORTED_SYMBOLS",
 ]
@@ -57,6 +58,9 @@ _SIGS = {
     "csa2_sparse_attn_workspace": (_SZ, [_I, _I, _I, _I, _I, _I]),
     "csa2_sparse_attn": (_I, [_I, _P, ctypes.POINTER(CSA2Kv), _P, _I, _I, _I, _I, _F, _P, _P, _P,
                               _SZ, _P]),
+    "csa2_index_scores_fp4": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I64, _P, _P, _I, _I, _P, _P]),
+    "csa2_index_topk_fp4": (_I, [_I, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I64, _P, _P, _I, _I, _P, _P,
+                                 _I, _I, _P, _SZ, _P]),
     "csa2_sparse_attn_swa_workspace": (_SZ, [_I, _I, _I, _I, _I, _I]),
     "csa2_sparse_attn_swa": (_I, [_I, _P, ctypes.POINTER(CSA2Kv), _P, _I, _I, _I, _I, _F, _P, _I64,
                                   _P, _I, _P, _P, _P, _SZ, _P]),
@@ -179,6 +183,45 @@ def csa2_index_scores(q, w, k, n_visible=None, pool=None, act: int = ACT_RELU, o
     _check(lib().csa2_index_scores(_ptr(q), _ptr(w), _ptr(k), B, Q, H, d, N, _ptr(n_visible),
                                    _ptr(pool), P, act, _ptr(out), _stream(stream)))
     return out
+
+
+def csa2_index_scores_fp4(q_codes, q_scales, w, k_codes, k_scales, n_visible=None, pool=None,
+                          act: int = ACT_RELU, out=None, stream=None):
+    """FP4 indexer: q codes/scales [B,Q,H,d/2]/[B,Q,H,d/16], K codes/scales
+    [B,N,d/2]/[B,N,d/16] (csa2_fp4_pack's format); returns bf16 scores."""
+    torch = _torch()
+    _need(q_codes, torch.uint8, 4, "q_codes")
+    _need(k_codes, torch.uint8, 3, "k_codes")
+    _need(w, torch.float32, 3, "w")
+    B, Q, H, d2 = q_codes.shape
+    N = k_codes.shape[1]
+    P = pool.shape[2] if pool is not None else 0
+    if out is None:
+        out = torch.empty(B, Q, P if pool is not None else N, dtype=torch.bfloat16, device=q_codes.device)
+    _check(lib().csa2_index_scores_fp4(_ptr(q_codes), _ptr(q_scales), _ptr(w), _ptr(k_codes),
+                                       _ptr(k_scales), B, Q, H, 2 * d2, N, _ptr(n_visible), _ptr(pool),
+                                       P, act, _ptr(out), _stream(stream)))
+    return out
+
+
+def csa2_index_topk_fp4(mode, q_codes, q_scales, w, k_codes, k_scales, k_top: int, n_visible=None,
+                        pool_in=None, pool_size: int = 0, act: int = ACT_RELU, stream=None):
+    """Scores (FP4 indexer, bf16) + selection for one Full / Reindex layer."""
+    torch = _torch()
+    mode = _MODE[mode]
+    B, Q, H, d2 = q_codes.shape
+    N = k_codes.shape[1]
+    P_in = pool_in.shape[2] if pool_in is not None else 0
+    topk = torch.empty(B, Q, k_top, dtype=torch.int32, device=q_codes.device)
+    pool = (torch.empty(B, Q, pool_size, dtype=torch.int32, device=q_codes.device)
+            if pool_size > 0 else None)
+    nb = lib().csa2_index_topk_workspace(B, Q, N, P_in, k_top, pool_size)
+    ws = _workspace(nb, q_codes.device)
+    _check(lib().csa2_index_topk_fp4(mode, _ptr(q_codes), _ptr(q_scales), _ptr(w), _ptr(k_codes),
+                                     _ptr(k_scales), B, Q, H, 2 * d2, N, _ptr(n_visible),
+                                     _ptr(pool_in), P_in, k_top, _ptr(topk), _ptr(pool), pool_size,
+                                     act, _ptr(ws), nb, _stream(stream)))
+    return topk, pool
 
 
 def _workspace(nbytes, device):

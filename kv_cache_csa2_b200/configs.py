@@ -44,6 +44,7 @@ class Workload:
     var_bias: float = 0.1
     var_attn_q: float = 1.0
     var_kv: float = 1.0
+    swa: int = 0                     # >0: every layer also attends its own window of this many uncompressed rows
 
     @property
     def N(self) -> int:
@@ -91,7 +92,12 @@ C5 = Workload(name="c5_prefill_4096_at_1m", B=1, Q=4096, L=1048576, m=4, D=512, 
               d=128, k=2048, modes=(FULL,) + (REUSE,) * 5, compress_new_tokens=4096, halo=True,
               q_pos0=1048576 - 4096, var_index_qk=1.0, w_dist=("normal", 1.0), var_bias=1.0)
 
-CONFIGS = {1: C1, 2: C2, 3: C3, 4: C4, 5: C5}
+# C6: C4 with the sliding-window branch the V4.1 layer layout gives every
+# layer: 128 uncompressed rows per layer and sequence, N(0,1) (not one of the
+# five benchmark workloads: the measurement of that branch at C4's scale).
+C6 = C4.replace(name="c6_hier_decode_swa128_1m", swa=128)
+
+CONFIGS = {1: C1, 2: C2, 3: C3, 4: C4, 5: C5, 6: C6}
 
 
 def n_visible(wl: Workload):

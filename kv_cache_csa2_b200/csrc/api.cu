@@ -443,6 +443,9 @@ csa2_status csa2_index_topk(csa2_mode mode, const void* q, const float* w, const
   if (!workspace || workspace_bytes < need)
     return fail(CSA2_ERR_OOM, "csa2_index_topk: workspace %zu < %zu bytes", workspace_bytes, need);
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  // many queries and no pool: scoring and selection in one kernel, no score round trip
+  if (!pool_in && !pool_out && index_topk_fused_applies(B, Q, H, d, N, k_top))
+    return launch_index_topk_fused(q, w, k, B, Q, H, d, N, n_visible, k_top, act, topk_out, s);
   float* scores = static_cast<float*>(workspace);
   const size_t sbytes = align256(static_cast<size_t>(rows) * L * sizeof(float));
   void* sel_ws = static_cast<char*>(workspace) + sbytes;
@@ -457,6 +460,86 @@ csa2_status csa2_index_topk(csa2_mode mode, const void* q, const float* w, const
   if (pool_out && clear.ptr && !clear.done) CSA2_TRY(select_topk_clear(rows, L, sel_ws, sel_bytes, s));
   if (pool_out) {
     // the pool and the top-k in the same selection passes when the kernel applies
+    const csa2_status st = launch_select_topk2(scores, rows, L, k_top, nullptr, topk_out, P_out,
+                                               pool_out, sel_ws, sel_bytes, s, true);
+    if (st != CSA2_ERR_UNSUPPORTED) return st;
+  }
+  CSA2_TRY(launch_select_topk(scores, rows, L, k_top, pool_in, topk_out, sel_ws, sel_bytes, s));
+  if (pool_out)
+    CSA2_TRY(launch_select_topk(scores, rows, L, P_out, nullptr, pool_out, sel_ws, sel_bytes, s));
+  return CSA2_OK;
+}
+
+// ------------------------------------------------------------- (a2, a3) FP4 indexer
+static csa2_status check_fp4_index_args(const char* fn, const uint8_t* q_codes,
+                                        const uint8_t* q_scales, const float* w,
+                                        const uint8_t* k_codes, const uint8_t* k_scales, int B,
+                                        int Q, int H, int d, int64_t N, const int32_t* pool, int P) {
+  if (B < 0 || Q < 0 || N < 0) return fail(CSA2_ERR_INVALID, "%s: negative size", fn);
+  if (H <= 0 || H > 64) return fail(CSA2_ERR_INVALID, "%s: H=%d outside [1, 64]", fn, H);
+  if (d != 64 && d != 128) return fail(CSA2_ERR_INVALID, "%s: d=%d must be 64 or 128", fn, d);
+  if (N > 0x7fffffffLL) return fail(CSA2_ERR_INVALID, "%s: N too large", fn);
+  if (pool && P <= 0) return fail(CSA2_ERR_INVALID, "%s: pool given with P=%d", fn, P);
+  if (B == 0 || Q == 0) return CSA2_OK;
+  const uintptr_t sal = static_cast<uintptr_t>(d / 16) - 1;   // scale rows: 8 or 4 bytes
+  if (!q_codes || !q_scales || !w || !k_codes || !k_scales || !aligned16(k_codes) ||
+      (reinterpret_cast<uintptr_t>(q_codes) & 7) || (reinterpret_cast<uintptr_t>(k_scales) & sal))
+    return fail(CSA2_ERR_INVALID,
+                "%s: null pointer, or k_codes not 16-byte, q_codes not 8-byte, k_scales not %d-byte aligned",
+                fn, d / 16);
+  return CSA2_OK;
+}
+
+csa2_status csa2_index_scores_fp4(const uint8_t* q_codes, const uint8_t* q_scales, const float* w,
+                                  const uint8_t* k_codes, const uint8_t* k_scales, int B, int Q,
+                                  int H, int d, int64_t N, const int32_t* n_visible,
+                                  const int32_t* pool, int P, csa2_index_act act, void* scores,
+                                  csa2_stream stream) {
+  CSA2_TRY(fault_gate());
+  CSA2_TRY(check_fp4_index_args(__func__, q_codes, q_scales, w, k_codes, k_scales, B, Q, H, d, N, pool, P));
+  if (B == 0 || Q == 0) return CSA2_OK;
+  REQUIRE(scores != nullptr, "csa2_index_scores_fp4: scores is null");
+  Fp4IndexArgs a{q_codes, q_scales, w, k_codes, k_scales, B, Q, H, d, N, n_visible, pool,
+                 pool ? P : 0, act, scores};
+  return launch_index_scores_fp4(a, true, reinterpret_cast<cudaStream_t>(stream));
+}
+
+csa2_status csa2_index_topk_fp4(csa2_mode mode, const uint8_t* q_codes, const uint8_t* q_scales,
+                                const float* w, const uint8_t* k_codes, const uint8_t* k_scales,
+                                int B, int Q, int H, int d, int64_t N, const int32_t* n_visible,
+                                const int32_t* pool_in, int P_in, int k_top, int32_t* topk_out,
+                                int32_t* pool_out, int P_out, csa2_index_act act, void* workspace,
+                                size_t workspace_bytes, csa2_stream stream) {
+  CSA2_TRY(fault_gate());
+  if (mode == CSA2_REUSE)
+    return fail(CSA2_ERR_MODE, "csa2_index_topk_fp4: a Reuse layer runs no indexer");
+  if (mode != CSA2_FULL && mode != CSA2_REINDEX)
+    return fail(CSA2_ERR_INVALID, "csa2_index_topk_fp4: unknown mode %d", int(mode));
+  if (mode == CSA2_FULL && pool_in)
+    return fail(CSA2_ERR_MODE, "csa2_index_topk_fp4: a Full layer builds its pool, pool_in must be NULL");
+  if (mode == CSA2_REINDEX && pool_out)
+    return fail(CSA2_ERR_MODE, "csa2_index_topk_fp4: a Reindex layer keeps no pool, pool_out must be NULL");
+  CSA2_TRY(check_fp4_index_args(__func__, q_codes, q_scales, w, k_codes, k_scales, B, Q, H, d, N,
+                                pool_in, P_in));
+  REQUIRE(k_top > 0, "csa2_index_topk_fp4: k_top=%d must be positive", k_top);
+  REQUIRE(!pool_out || P_out > 0, "csa2_index_topk_fp4: pool_out given with P_out=%d", P_out);
+  if (B == 0 || Q == 0) return CSA2_OK;
+  REQUIRE(topk_out != nullptr, "csa2_index_topk_fp4: topk_out is null");
+  const int64_t L = pool_in ? P_in : N;
+  const int64_t rows = static_cast<int64_t>(B) * Q;
+  const size_t need = csa2_index_topk_workspace(B, Q, N, pool_in ? P_in : 0, k_top, pool_out ? P_out : 0);
+  if (!workspace || workspace_bytes < need)
+    return fail(CSA2_ERR_OOM, "csa2_index_topk_fp4: workspace %zu < %zu bytes", workspace_bytes, need);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  float* scores = static_cast<float*>(workspace);          // f32 holding bf16 values
+  const size_t sbytes = align256(static_cast<size_t>(rows) * L * sizeof(float));
+  void* sel_ws = static_cast<char*>(workspace) + sbytes;
+  const size_t sel_bytes = workspace_bytes - sbytes;
+  Fp4IndexArgs a{q_codes, q_scales, w, k_codes, k_scales, B, Q, H, d, N, n_visible, pool_in,
+                 pool_in ? P_in : 0, act, scores};
+  CSA2_TRY(launch_index_scores_fp4(a, false, s));
+  if (pool_out) {
+    CSA2_TRY(select_topk_clear(rows, L, sel_ws, sel_bytes, s));
     const csa2_status st = launch_select_topk2(scores, rows, L, k_top, nullptr, topk_out, P_out,
                                                pool_out, sel_ws, sel_bytes, s, true);
     if (st != CSA2_ERR_UNSUPPORTED) return st;

@@ -34,14 +34,26 @@ struct AttnSmem {
                                   3 * HA * 4 + 2 * kR * 4;
 };
 
-// The row sources of launch_sparse_attn (AttnRows) as the kernel takes them.
+// The row sources of launch_sparse_attn (AttnRows) as the kernel takes them,
+// and the split of a query's rows over CTAs.
 struct SimtRows {
   const int32_t* n_visible;
   const uint16_t* win;
   int64_t win_rows;
   const int32_t* win_end;
   int W;
+  int Q;              // queries per sequence
+  int64_t q_base;     // first query (flat b * Q + q) of this launch
+  int n_chunks;       // CTAs per query; 1: one CTA takes every row and writes the output
+  int chunk_rows;     // rows (slots) per CTA, a multiple of kR
+  float* part;        // [queries of the launch][n_chunks][HA * DD + 2 HA]: sums, max, row sum
+  unsigned* counters; // [queries of the launch], zero before the launch, left zero after it
 };
+
+// weight of a partial with max m in a sum whose max is M (0 for empty partials)
+__device__ __forceinline__ float rescale_part(float m, float M) {
+  return (m == -INFINITY || M == -INFINITY) ? 0.0f : expf(m - M);
+}
 
 template <int HA, int DD, bool FP4>
 __global__ void __launch_bounds__(kT) attn_simt_kernel(
@@ -63,9 +75,12 @@ __global__ void __launch_bounds__(kT) attn_simt_kernel(
   int* id_s = reinterpret_cast<int*>(a_s + HA);   // [kR] row ids; [kR] their source (1 = window)
   int* src_s = id_s + kR;
 
+  __shared__ int last_s;
   const int tid = threadIdx.x;
-  const int64_t seq = blockIdx.y;                                   // sequence b
-  const int64_t qi = seq * gridDim.x + blockIdx.x;                  // flat (b, q)
+  const int64_t ql = blockIdx.x / rs.n_chunks;                      // query within the launch
+  const int chunk = static_cast<int>(blockIdx.x % rs.n_chunks);
+  const int64_t qi = rs.q_base + ql;                                // flat (b, q)
+  const int64_t seq = qi / rs.Q;                                    // sequence b
   const uint32_t* qg = reinterpret_cast<const uint32_t*>(q + qi * HA * DD);
   for (int i = tid; i < HA * DD / 2; i += kT) q_s[i] = qg[i];
   for (int h = tid; h < HA; h += kT) { m_s[h] = -INFINITY; l_s[h] = 0.0f; }
@@ -84,21 +99,25 @@ __global__ void __launch_bounds__(kT) attn_simt_kernel(
       w_end = 0;
     }
   }
-  const int slots = k + (rs.win ? rs.W : 0);
+  // this CTA's slots: [chunk * chunk_rows, +chunk_rows) of the query's
+  // k selected and W window slots
+  const int slots = min(k + (rs.win ? rs.W : 0), (chunk + 1) * rs.chunk_rows);
 
-  for (int c0 = 0; c0 < slots; c0 += kR) {
+  for (int c0 = chunk * rs.chunk_rows; c0 < slots; c0 += kR) {
     __syncthreads();   // previous step done with rows_s / p_s / id_s
     if (tid < kR) {
       const int s = c0 + tid;
       int id = -1, src = 0;
-      if (s < k) {
+      if (s >= slots) {
+        // past this CTA's slots
+      } else if (s < k) {
         if (topk) {
           id = topk[qi * k + s];
           if (id >= n || id < -1) { raise_dev_error(err, DEVERR_BOUNDS); id = -1; }
         } else {
           id = s < vis ? s : -1;
         }
-      } else if (s < slots) {
+      } else {
         const int row = w_end - rs.W + (s - k);
         id = row >= 0 ? row : -1;
         src = 1;
@@ -218,40 +237,141 @@ __global__ void __launch_bounds__(kT) attn_simt_kernel(
     }
   }
   __syncthreads();
-  const float l = l_s[h_o];
-  const float inv = l > 0.0f ? 1.0f / l : 0.0f;
   uint16_t* og = out + (qi * HA + h_o) * DD + d_o;
+  if (rs.n_chunks <= 1) {
+    const float l = l_s[h_o];
+    const float inv = l > 0.0f ? 1.0f / l : 0.0f;
+#pragma unroll
+    for (int i = 0; i < OPT; ++i) {
+      __nv_bfloat16 v = __float2bfloat16_rn(acc[i] * inv);
+      og[i * TPH] = *reinterpret_cast<uint16_t*>(&v);
+    }
+    if (lse && d_o == 0) lse[qi * HA + h_o] = l > 0.0f ? m_s[h_o] + logf(l) : -INFINITY;
+    return;
+  }
+  // this chunk's partial: unnormalised sums, the running max and row sum per head
+  constexpr int kStride = HA * DD + 2 * HA;
+  float* pp = rs.part + (ql * rs.n_chunks + chunk) * kStride;
+#pragma unroll
+  for (int i = 0; i < OPT; ++i) __stcg(pp + h_o * DD + d_o + i * TPH, acc[i]);
+  for (int h = tid; h < HA; h += kT) {
+    __stcg(pp + HA * DD + h, m_s[h]);
+    __stcg(pp + HA * DD + HA + h, l_s[h]);
+  }
+  __threadfence();
+  __syncthreads();
+  if (tid == 0) last_s = atomicAdd(rs.counters + ql, 1u) == static_cast<unsigned>(rs.n_chunks - 1);
+  __syncthreads();
+  if (!last_s) return;
+  // the query's last chunk to finish combines the partials, in chunk order
+  __threadfence();
+  const float* pq = rs.part + ql * rs.n_chunks * kStride;
+  float M = -INFINITY;
+  for (int c = 0; c < rs.n_chunks; ++c) M = fmaxf(M, __ldcg(pq + c * kStride + HA * DD + h_o));
+  float L = 0.0f, o[OPT];
+#pragma unroll
+  for (int i = 0; i < OPT; ++i) o[i] = 0.0f;
+  for (int c = 0; c < rs.n_chunks; ++c) {
+    const float* pc = pq + c * kStride;
+    const float wc = rescale_part(__ldcg(pc + HA * DD + h_o), M);
+    L += __ldcg(pc + HA * DD + HA + h_o) * wc;
+#pragma unroll
+    for (int i = 0; i < OPT; ++i) o[i] += __ldcg(pc + h_o * DD + d_o + i * TPH) * wc;
+  }
+  const float inv = L > 0.0f ? 1.0f / L : 0.0f;
 #pragma unroll
   for (int i = 0; i < OPT; ++i) {
-    __nv_bfloat16 v = __float2bfloat16_rn(acc[i] * inv);
+    __nv_bfloat16 v = __float2bfloat16_rn(o[i] * inv);
     og[i * TPH] = *reinterpret_cast<uint16_t*>(&v);
   }
-  if (lse && d_o == 0) lse[qi * HA + h_o] = l > 0.0f ? m_s[h_o] + logf(l) : -INFINITY;
+  if (lse && d_o == 0) lse[qi * HA + h_o] = L > 0.0f ? M + logf(L) : -INFINITY;
+  if (tid == 0) rs.counters[ql] = 0u;            // ready for the next launch
+}
+
+// The split of a query's slots over CTAs: it depends on the slots alone (k and
+// the window), so a query's result does not depend on the batch.  Up to
+// kMaxChunks CTAs of at least kR rows each.
+constexpr int kMaxChunks = 16;
+constexpr size_t kSimtWsCap = size_t(64) << 20;   // partials of one launch
+struct Split {
+  int n_chunks, chunk_rows;
+  int64_t per_launch;                             // queries per launch (partials in the workspace)
+  size_t bytes;                                   // workspace: partials, then counters
+};
+
+Split split_for(int64_t n_queries, int Ha, int D, int k, bool win, int W) {
+  Split s;
+  const int slots = k + (win ? W : 0);
+  s.n_chunks = slots <= kR ? 1 : std::min(kMaxChunks, (slots + kR - 1) / kR);
+  const int per = (slots + s.n_chunks - 1) / s.n_chunks;
+  s.chunk_rows = std::max(kR, (per + kR - 1) / kR * kR);
+  s.n_chunks = std::max(1, (slots + s.chunk_rows - 1) / s.chunk_rows);
+  if (s.n_chunks == 1) {
+    s.per_launch = n_queries;
+    s.bytes = 0;
+    return s;
+  }
+  const size_t per_query = static_cast<size_t>(s.n_chunks) * (static_cast<size_t>(Ha) * D + 2 * Ha) * 4;
+  s.per_launch = std::max<int64_t>(1, std::min<int64_t>(n_queries, static_cast<int64_t>(kSimtWsCap / per_query)));
+  s.bytes = ((static_cast<size_t>(s.per_launch) * per_query + 255) & ~size_t(255)) +
+            ((static_cast<size_t>(s.per_launch) * 4 + 255) & ~size_t(255));
+  return s;
 }
 
 template <int HA, int DD>
 csa2_status run_simt(const void* q, const csa2_kv& kv, const int32_t* topk, int B, int Q, int k,
-                     float scale, void* out, float* lse, cudaStream_t stream, const AttnRows& rows) {
+                     float scale, void* out, float* lse, void* ws, size_t ws_bytes,
+                     unsigned long long* sync_zeroed, cudaStream_t stream, const AttnRows& rows) {
   const size_t smem = AttnSmem<HA, DD>::bytes;
   auto kern = kv.fmt == CSA2_KV_FP4 ? attn_simt_kernel<HA, DD, true> : attn_simt_kernel<HA, DD, false>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            static_cast<int>(smem)) != cudaSuccess)
     return check_launch("sparse_attn: shared-memory opt-in");
-  if (B > 65535) return fail(CSA2_ERR_UNSUPPORTED, "sparse_attn: B > 65535");
-  begin_launch(stream);
-  kern<<<dim3(static_cast<unsigned>(Q), static_cast<unsigned>(B)), kT, smem, stream>>>(
-      static_cast<const uint16_t*>(q), kv.data, kv.scales, kv.n, topk, k, scale,
-      static_cast<uint16_t*>(out), lse, device_error_word(),
-      SimtRows{rows.n_visible, static_cast<const uint16_t*>(rows.win), rows.win_rows, rows.win_end,
-               rows.win ? rows.W : 0});
-  note_launch(LK_ATTN, 1, stream);
-  return check_launch("sparse_attn");
+  const int64_t n_queries = static_cast<int64_t>(B) * Q;
+  Split sp = split_for(n_queries, HA, DD, k, rows.win != nullptr, rows.W);
+  if (sp.n_chunks > 1 && (!ws || ws_bytes < sp.bytes)) {     // no room for partials: one CTA per query
+    sp.n_chunks = 1;
+    sp.chunk_rows = k + (rows.win ? rows.W : 0);
+    sp.per_launch = n_queries;
+  }
+  SimtRows rs{rows.n_visible, static_cast<const uint16_t*>(rows.win), rows.win_rows, rows.win_end,
+              rows.win ? rows.W : 0, Q, 0, sp.n_chunks, std::max(sp.chunk_rows, 1), nullptr, nullptr};
+  // the counters: a layer group's (zeroed once, left zero by every launch)
+  // when they are enough, else the workspace's, cleared before each launch
+  const bool own_counters = !(sync_zeroed && sp.per_launch <= 2 * kAttnMaxGrid);
+  if (sp.n_chunks > 1) {
+    const size_t part_bytes = sp.bytes - ((static_cast<size_t>(sp.per_launch) * 4 + 255) & ~size_t(255));
+    rs.part = static_cast<float*>(ws);
+    rs.counters = own_counters ? reinterpret_cast<unsigned*>(static_cast<char*>(ws) + part_bytes)
+                               : reinterpret_cast<unsigned*>(sync_zeroed);
+  }
+  for (int64_t q0 = 0; q0 < n_queries; q0 += sp.per_launch) {
+    const int64_t nq = std::min<int64_t>(sp.per_launch, n_queries - q0);
+    const int64_t grid = nq * sp.n_chunks;
+    if (grid > 0x7fffffffLL) return fail(CSA2_ERR_UNSUPPORTED, "sparse_attn: too many CTAs");
+    rs.q_base = q0;
+    if (sp.n_chunks > 1 && own_counters) {
+      begin_launch(stream);
+      if (cudaMemsetAsync(rs.counters, 0, static_cast<size_t>(nq) * 4, stream) != cudaSuccess)
+        return check_launch("sparse_attn: clear counters");
+      note_launch(LK_OTHER, 1, stream);
+    }
+    begin_launch(stream);
+    kern<<<static_cast<unsigned>(grid), kT, smem, stream>>>(
+        static_cast<const uint16_t*>(q), kv.data, kv.scales, kv.n, topk, k, scale,
+        static_cast<uint16_t*>(out), lse, device_error_word(), rs);
+    note_launch(LK_ATTN, 1, stream);
+    CSA2_TRY(check_launch("sparse_attn"));
+  }
+  return CSA2_OK;
 }
 
 }  // namespace
 
 size_t sparse_attn_workspace(int B, int Q, int Ha, int D, int k, csa2_kv_fmt fmt, bool window) {
-  return sparse_attn_tc_workspace(B, Q, Ha, D, k, fmt, window);
+  const size_t tc = sparse_attn_tc_workspace(B, Q, Ha, D, k, fmt, window);
+  if (tc > 0) return tc;
+  return split_for(static_cast<int64_t>(B) * Q, Ha, D, k, window, kMaxWindow).bytes;
 }
 
 csa2_status launch_sparse_attn(const void* q, const csa2_kv& kv, const int32_t* topk, int B,
@@ -263,12 +383,12 @@ csa2_status launch_sparse_attn(const void* q, const csa2_kv& kv, const int32_t* 
                                         sync_zeroed, stream, rows);
   if (s != CSA2_ERR_UNSUPPORTED) return s;
   const int D = kv.dim;
-  if (Ha == 64 && D == 512) return run_simt<64, 512>(q, kv, topk, B, Q, k, scale, out, lse, stream, rows);
-  if (Ha == 16 && D == 128) return run_simt<16, 128>(q, kv, topk, B, Q, k, scale, out, lse, stream, rows);
-  if (Ha == 16 && D == 512) return run_simt<16, 512>(q, kv, topk, B, Q, k, scale, out, lse, stream, rows);
-  if (Ha == 64 && D == 128) return run_simt<64, 128>(q, kv, topk, B, Q, k, scale, out, lse, stream, rows);
-  if (Ha == 32 && D == 128) return run_simt<32, 128>(q, kv, topk, B, Q, k, scale, out, lse, stream, rows);
-  if (Ha == 32 && D == 512) return run_simt<32, 512>(q, kv, topk, B, Q, k, scale, out, lse, stream, rows);
+#define CSA2_SIMT(HA_, D_)                                                                       \
+  if (Ha == HA_ && D == D_)                                                                      \
+    return run_simt<HA_, D_>(q, kv, topk, B, Q, k, scale, out, lse, ws, ws_bytes, sync_zeroed, stream, rows);
+  CSA2_SIMT(64, 512) CSA2_SIMT(16, 128) CSA2_SIMT(16, 512) CSA2_SIMT(64, 128) CSA2_SIMT(32, 128)
+  CSA2_SIMT(32, 512)
+#undef CSA2_SIMT
   return fail(CSA2_ERR_UNSUPPORTED, "sparse_attn: (Ha=%d, D=%d) not instantiated", Ha, D);
 }
 

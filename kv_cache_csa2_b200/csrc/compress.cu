@@ -78,25 +78,44 @@ __global__ void __launch_bounds__(256) compress_kernel(
 // HCA compression ("读完这篇，你就搞懂 DeepSeek v4 了", HCA 压缩机制, eq. 10 and
 // 11): entry j is the per-channel softmax-weighted sum of the m tokens of
 // block j alone (no overlap with the block before), bias [m, D] indexed by the
-// position in the block.  Blocks are long (m up to 1024), so each thread runs
-// one pass over its block with a running max (the sums are rescaled when the
-// max grows) instead of the two passes of the overlapping kernel.
+// position in the block.  Blocks are long (m up to 1024), so the block's rows
+// are split over kHcaSplit lanes of a warp (lane s takes rows s, s + 8, ..),
+// each lane runs one pass with a running max (its sums rescaled when the max
+// grows), and the lanes' (max, sum, weighted sum) merge by shuffles in a fixed
+// order.  A warp covers 4 channel groups (128 bytes of z) of 8 rows at a time.
+constexpr int kHcaSplit = 8;
+
+__device__ __forceinline__ void merge_softmax(float& mx, float& den, float& num, float mx2, float den2,
+                                              float num2) {
+  const float M = fmaxf(mx, mx2);
+  const float a = mx == -INFINITY ? 0.0f : expf(mx - M);
+  const float b = mx2 == -INFINITY ? 0.0f : expf(mx2 - M);
+  den = den * a + den2 * b;
+  num = num * a + num2 * b;
+  mx = M;
+}
+
 __global__ void __launch_bounds__(256) compress_hca_kernel(
     const uint16_t* __restrict__ c, const float* __restrict__ z, const float* __restrict__ bias,
     int N, int D, int m, int64_t t_in, uint16_t* __restrict__ out, int64_t out_bstride) {
   const int groups = D / 8;
-  const int64_t gid = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x;
+  const int64_t tid = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x;
+  const int lane = threadIdx.x & 31;
+  const int s = lane / 4;                          // this lane's share of the rows: s, s + 8, ...
+  // (entry, channel group) of the lane: 4 per warp, consecutive channel groups
+  const int64_t gid = (tid / 32) * 4 + (lane & 3);
   const int b = blockIdx.y;
-  if (gid >= static_cast<int64_t>(N) * groups) return;
-  const int j = static_cast<int>(gid / groups);
-  const int ch0 = static_cast<int>(gid % groups) * 8;
+  const bool live = gid < static_cast<int64_t>(N) * groups;
+  const int j = live ? static_cast<int>(gid / groups) : 0;
+  const int ch0 = live ? static_cast<int>(gid % groups) * 8 : 0;
   const int64_t seq = static_cast<int64_t>(b) * t_in * D;
   const int64_t first = static_cast<int64_t>(j) * m;
 
   float mx[8], den[8], num[8];
 #pragma unroll
   for (int u = 0; u < 8; ++u) { mx[u] = -INFINITY; den[u] = 0.0f; num[u] = 0.0f; }
-  for (int w = 0; w < m; ++w) {
+#pragma unroll 2
+  for (int w = s; w < (live ? m : 0); w += kHcaSplit) {
     float zz[8], bb[8];
     load8f(z + seq + (first + w) * D + ch0, zz);
     load8f(bias + static_cast<int64_t>(w) * D + ch0, bb);
@@ -117,6 +136,18 @@ __global__ void __launch_bounds__(256) compress_hca_kernel(
       num[u] = fmaf(p, cc[u], num[u]);
     }
   }
+  // the 8 lanes of one (entry, channel group) sit 4 apart: merge them
+#pragma unroll
+  for (int ofs = 16; ofs >= 4; ofs >>= 1) {
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const float mx2 = __shfl_xor_sync(0xffffffffu, mx[u], ofs);
+      const float den2 = __shfl_xor_sync(0xffffffffu, den[u], ofs);
+      const float num2 = __shfl_xor_sync(0xffffffffu, num[u], ofs);
+      merge_softmax(mx[u], den[u], num[u], mx2, den2, num2);
+    }
+  }
+  if (!live || s != 0) return;
   uint4 o;
   o.x = pack_bf16x2(num[0] / den[0], num[1] / den[1]);
   o.y = pack_bf16x2(num[2] / den[2], num[3] / den[3]);
@@ -132,9 +163,10 @@ csa2_status launch_compress_hca(const void* c, const float* z, const float* bias
                                 int D, int m, void* out, int64_t out_bstride, cudaStream_t stream) {
   const int64_t N = T / m;
   if (N == 0 || B == 0) return CSA2_OK;
-  const int64_t work = N * (D / 8);
+  const int64_t work = N * (D / 8);                  // (entry, channel group) pairs, 4 per warp
+  const int64_t lanes = (work + 3) / 4 * 32;
   const int threads = 256;
-  dim3 grid(static_cast<unsigned>((work + threads - 1) / threads), static_cast<unsigned>(B));
+  dim3 grid(static_cast<unsigned>((lanes + threads - 1) / threads), static_cast<unsigned>(B));
   begin_launch(stream);
   compress_hca_kernel<<<grid, threads, 0, stream>>>(static_cast<const uint16_t*>(c), z, bias,
                                                     static_cast<int>(N), D, m, T,

@@ -28,6 +28,33 @@ csa2_status launch_index_scores(const void* q, const float* w, const void* k, in
                                 int P, csa2_index_act act, float* scores, cudaStream_t stream,
                                 ClearOnLaunch* clear = nullptr);
 
+// A Full layer's indexer fused with a streaming top-k (no score round trip):
+// many queries (at least one group of 4 per SM), k_top <= kMaxFusedTopk.
+// Same scores and the same exact selection as scoring then selecting.
+constexpr int kMaxFusedTopk = 2048;
+bool index_topk_fused_applies(int B, int Q, int H, int d, int64_t N, int k_top);
+csa2_status launch_index_topk_fused(const void* q, const float* w, const void* k, int B, int Q,
+                                    int H, int d, int64_t N, const int32_t* n_visible, int k_top,
+                                    csa2_index_act act, int32_t* topk, cudaStream_t stream);
+
+// FP4 indexer (q and K in the main-KV FP4 format, bf16 scores): scores
+// rounded to bf16, stored as bf16 (out_bf16) or as f32 holding the bf16 value.
+struct Fp4IndexArgs {
+  const uint8_t* q_codes;    // [B, Q, H, d/2]
+  const uint8_t* q_scales;   // [B, Q, H, d/16]
+  const float* w;            // [B, Q, H]
+  const uint8_t* k_codes;    // [B, N, d/2]
+  const uint8_t* k_scales;   // [B, N, d/16]
+  int B, Q, H, d;
+  int64_t N;
+  const int32_t* n_visible;  // [B, Q] or null
+  const int32_t* pool;       // [B, Q, P] or null
+  int P;
+  csa2_index_act act;
+  void* scores;              // [B, Q, N or P]
+};
+csa2_status launch_index_scores_fp4(const Fp4IndexArgs& a, bool out_bf16, cudaStream_t stream);
+
 size_t select_topk_workspace(int64_t rows, int64_t L, int count);
 // The workspace one selection (launch_select_topk) will actually use on the
 // current device: 0 when the cluster, one-CTA or fallback kernel takes the

@@ -137,6 +137,9 @@ def make_layer_inputs(wl: Workload, i: int, seed: int = 0) -> dict:
     nm = wl.name
     mode = wl.modes[i]
     L = {"q_attn": normal_bf16(_rng(seed, nm, 100 + 10 * i), (wl.B, wl.Q, wl.Ha, wl.D), wl.var_attn_q)}
+    if wl.swa:       # this layer's own window rows: the last swa tokens, every query sees all of them
+        L["win"] = normal_bf16(_rng(seed, nm, 103 + 10 * i), (wl.B, wl.swa, wl.D), wl.var_kv)
+        L["win_end"] = np.full((wl.B, wl.Q), wl.swa, dtype=np.int32)
     if mode in (FULL, REINDEX):
         var = wl.index_var if mode == FULL else wl.reindex_var
         L["q_index"] = normal_bf16(_rng(seed, nm, 101 + 10 * i), (wl.B, wl.Q, wl.Hi, wl.d), var)

@@ -38,13 +38,14 @@ def bf16_ulp(x):
     return np.where(ax >= 2.0 ** -126, np.ldexp(1.0, (e - 7).astype(int)), 2.0 ** -133)
 
 
-def check_selection(gpu_row, cand_ids, cand_scores, k, what=""):
+def check_selection(gpu_row, cand_ids, cand_scores, k, what="", tie_tol=None):
     """GPU top-k row (entry ids) against the oracle's scores of the candidates.
 
     The GPU set must be a valid selection (ascending, unique, candidates only,
     -1 padded, min(k, selectable) long).  It must equal the oracle's set except
     for entries whose oracle score lies within TIE_REL*|s_k| (floor TIE_ABS) of
-    the oracle's k-th score s_k.  Returns True when the sets are identical.
+    the oracle's k-th score s_k -- or within tie_tol(s_k) when given (bf16
+    scores: one bf16 step).  Returns True when the sets are identical.
     """
     cand_ids = np.asarray(cand_ids)
     ok = cand_scores > -np.inf
@@ -60,7 +61,7 @@ def check_selection(gpu_row, cand_ids, cand_scores, k, what=""):
         return True
     opos = O.select_top(cand_scores[None], k)[0][:n]
     s_k = cand_scores[opos].min()
-    tol = max(TIE_REL * abs(s_k), TIE_ABS)
+    tol = max(TIE_REL * abs(s_k), TIE_ABS) if tie_tol is None else float(tie_tol(s_k))
     g_only = np.setdiff1d(pos, opos)
     o_only = np.setdiff1d(opos, pos)
     assert np.all(cand_scores[g_only] >= s_k - tol), f"{what}: GPU pick below the tie band"

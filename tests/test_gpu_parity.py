@@ -412,9 +412,12 @@ def test_reuse_runs_no_indexer_and_mode_order():
     g.close()
 
 
-def test_batch_invariance_bitwise():
-    """A query's selection and output do not depend on the batch it runs in."""
-    wl = SMALL[3]
+@pytest.mark.parametrize("which", [3, 2], ids=["tensor_core_attn", "split_cuda_core_attn_fp4"])
+def test_batch_invariance_bitwise(which):
+    """A query's selection and output do not depend on the batch it runs in
+    (the tensor-core attention of 64 x 512 heads, and the split CUDA-core
+    attention of 16 x 128 heads over FP4 entries)."""
+    wl = SMALL[which]
     inp = I.make_inputs(wl, seed=14)
     full, _ = U.gpu_group(wl, inp)
     for b in range(wl.B):
