@@ -5,12 +5,14 @@
 // is the main-KV one of "Recall之王" (E2M1 values, one E4M3 scale per 16
 // channels).
 //
-// An E2M1 value times an E4M3 scale has at most 6 significant bits, so every
-// dequantised q and K value is exact in bf16 and every product q_i k_i is
-// exact in f32: the contraction runs as the bf16 kernel's (tcgen05 kind::f16,
-// f32 accumulation) on tiles dequantised in shared memory, and only the bytes
-// read from memory shrink (72 instead of 256 per 128-wide key row).  Each
-// score is rounded once to bf16.
+// An E2M1 value times an E4M3 scale has at most 6 significant bits and lies
+// in [2^-10, 2688], so every dequantised q and K value is exact in f16 (the
+// hardware E2M1 -> f16 conversion, then one exact multiply by the scale) and
+// every product q_i k_i is exact in f32: the contraction runs on the tensor
+// cores (tcgen05 kind::f16 with f16 operands, f32 accumulation) on tiles
+// dequantised in shared memory, and only the bytes read from memory shrink
+// (72 instead of 256 per 128-wide key row).  Each score is rounded once to
+// bf16.
 //
 // Per CTA (persistent, one per SM), units = (query, tile of 128 keys) in a
 // contiguous range:
@@ -79,8 +81,8 @@ struct Cfg {
   static constexpr int OFF_Q = OFF_A + STAGES * TILE_A;
   static constexpr int OFF_RAW = OFF_Q + 2 * QBYTES;
   static constexpr int OFF_W = OFF_RAW + kRaw * RAW_SLOT;
-  static constexpr int OFF_LUT = OFF_W + 2 * HP * 4;        // [256] byte -> two E2M1 values (bf16)
-  static constexpr int OFF_BAR = OFF_LUT + 256 * 4;
+
+  static constexpr int OFF_BAR = OFF_W + 2 * HP * 4;
   static constexpr int NBAR = 2 * STAGES + 9;      // + the teardown barrier
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
   static constexpr int BYTES = OFF_MISC + 16 + 1024;
@@ -97,22 +99,26 @@ __device__ __forceinline__ float e4m3_to_f32(uint32_t c) {
   return (c & 128u) ? -mag : mag;
 }
 
+// Two E2M1 codes (one byte: the lower channel in the low nibble) -> f16x2
+// (lower channel in the low half), by the hardware conversion.
+__device__ __forceinline__ uint32_t e2m1x2_to_f16x2(uint32_t byte) {
+  uint32_t r;
+  const uint16_t b = static_cast<uint16_t>(byte);
+  asm("{\n\t.reg .b8 t;\n\tcvt.u8.u16 t, %1;\n\tcvt.rn.f16x2.e2m1x2 %0, t;\n\t}" : "=r"(r) : "h"(b));
+  return r;
+}
+
 // One 16-channel block: 8 code bytes (channel 2i low nibble, 2i+1 high) and
-// its scale -> 8 words of two bf16 each (exact).
-__device__ __forceinline__ void fp4_block_to_bf16(uint2 codes, uint32_t scale, uint32_t (&out)[8]) {
-  const float s = e4m3_to_f32(scale);
+// its E4M3 scale -> 8 words of two f16 each.  Exact: an E2M1 value times an
+// E4M3 scale has at most 6 significant bits and lies in [2^-10, 2688].
+__device__ __forceinline__ void fp4_block_to_f16(uint2 codes, uint32_t scale, uint32_t (&out)[8]) {
+  const __half sh = __float2half_rn(e4m3_to_f32(scale));
+  const __half2 s2 = __halves2half2(sh, sh);
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
-    const uint32_t byte = ((i < 4 ? codes.x : codes.y) >> (8 * (i & 3))) & 0xffu;
-    float v[2];
-#pragma unroll
-    for (int t = 0; t < 2; ++t) {
-      const uint32_t c = (byte >> (4 * t)) & 15u;
-      const uint32_t e = (c >> 1) & 3u, mt = c & 1u;
-      const float mag = e == 0 ? 0.5f * mt : (1.0f + 0.5f * mt) * static_cast<float>(1u << (e - 1));
-      v[t] = ((c & 8u) ? -mag : mag) * s;
-    }
-    out[i] = pack_bf16x2(v[0], v[1]);
+    const uint32_t pr = e2m1x2_to_f16x2(((i < 4 ? codes.x : codes.y) >> (8 * (i & 3))) & 0xffu);
+    const __half2 v = __hmul2(*reinterpret_cast<const __half2*>(&pr), s2);
+    out[i] = *reinterpret_cast<const uint32_t*>(&v);
   }
 }
 
@@ -126,7 +132,7 @@ __global__ void __launch_bounds__(kThreads, 1) index_fp4_kernel(const Params p) 
   uint8_t* sQ = smem + C::OFF_Q;
   uint8_t* sRaw = smem + C::OFF_RAW;
   float* sW = reinterpret_cast<float*>(smem + C::OFF_W);
-  uint32_t* sLut = reinterpret_cast<uint32_t*>(smem + C::OFF_LUT);
+
   uint64_t* bar = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
   uint64_t* full = bar;                      // [S] a bf16 key tile is ready (128 loader arrivals)
   uint64_t* empty = bar + S;                 // [S] the MMAs of a tile are done
@@ -188,7 +194,7 @@ __global__ void __launch_bounds__(kThreads, 1) index_fp4_kernel(const Params p) 
         if (h < p.H) {
           const int64_t hr = qrow * p.H + h;
           const uint2 cw = __ldg(reinterpret_cast<const uint2*>(p.q_codes + hr * (DK / 2)) + blk);
-          fp4_block_to_bf16(cw, __ldg(p.q_scales + hr * NBLK + blk), o);
+          fp4_block_to_f16(cw, __ldg(p.q_scales + hr * NBLK + blk), o);
         }
         const int kb = blk / 4, c = (blk % 4) * 2;
         *reinterpret_cast<uint4*>(qs + kb * C::QKB + sw128_offset(h, c)) = make_uint4(o[0], o[1], o[2], o[3]);
@@ -202,7 +208,7 @@ __global__ void __launch_bounds__(kThreads, 1) index_fp4_kernel(const Params p) 
   } else if (warp == 1) {
     // ---------------------------------------------------------------- MMA issuer
     if (lane == 0) {
-      constexpr uint32_t idesc = idesc_bf16_f32(128, HP, false, false);
+      constexpr uint32_t idesc = idesc_f16_f32(128, HP, false, false);
       int64_t prev = -1;
       int qi = -1;
       int64_t it = 0;
@@ -272,16 +278,6 @@ __global__ void __launch_bounds__(kThreads, 1) index_fp4_kernel(const Params p) 
     // the 128 loader threads dequantise a tile together, once each has seen its
     // own copies land (named barrier 3): thread r takes 16-channel blocks
     // r + 128 u, so eight threads read one row's codes contiguously
-    for (int i = r; i < 256; i += 128) {              // byte -> two unscaled E2M1 values in bf16
-      uint32_t pr = 0;
-#pragma unroll
-      for (int t = 0; t < 2; ++t) {
-        const uint32_t c = (static_cast<uint32_t>(i) >> (4 * t)) & 15u;
-        const uint32_t mags[8] = {0x0000u, 0x3F00u, 0x3F80u, 0x3FC0u, 0x4000u, 0x4040u, 0x4080u, 0x40C0u};
-        pr |= (mags[c & 7u] | ((c & 8u) ? 0x8000u : 0u)) << (16 * t);
-      }
-      sLut[i] = pr;
-    }
     auto load_bar = [] { asm volatile("bar.sync 3, 128;" ::: "memory"); };
     auto convert = [&](int64_t it_c) {
       const int stage = static_cast<int>(it_c % S);
@@ -296,15 +292,8 @@ __global__ void __launch_bounds__(kThreads, 1) index_fp4_kernel(const Params p) 
       for (int u = 0; u < NBLK; ++u) {
         const int i = r + 128 * u, row = i / NBLK, blk = i % NBLK;
         const uint2 cw = *reinterpret_cast<const uint2*>(src + row * (DK / 2) + 8 * blk);
-        const __nv_bfloat16 sb = __float2bfloat16_rn(e4m3_to_f32(src[C::RAW_CODES + row * NBLK + blk]));
-        const __nv_bfloat162 s2 = __halves2bfloat162(sb, sb);
         uint32_t o[8];
-#pragma unroll
-        for (int t = 0; t < 8; ++t) {               // exact: at most 6 significant bits
-          const uint32_t pr = sLut[((t < 4 ? cw.x : cw.y) >> (8 * (t & 3))) & 0xffu];
-          const __nv_bfloat162 v = __hmul2(*reinterpret_cast<const __nv_bfloat162*>(&pr), s2);
-          o[t] = *reinterpret_cast<const uint32_t*>(&v);
-        }
+        fp4_block_to_f16(cw, src[C::RAW_CODES + row * NBLK + blk], o);
         const int kb = blk / 4, c = (blk % 4) * 2;
         *reinterpret_cast<uint4*>(dst + kb * kKBlockBytes + sw128_offset(row, c)) = make_uint4(o[0], o[1], o[2], o[3]);
         *reinterpret_cast<uint4*>(dst + kb * kKBlockBytes + sw128_offset(row, c + 1)) = make_uint4(o[4], o[5], o[6], o[7]);

@@ -41,7 +41,7 @@ constexpr int kPoolThreads = 13 * 32;
 constexpr int kPoolRows = 128 * 8 / kPoolProducers;   // rows per producer thread and tile
 constexpr int kTileRows = 128;
 constexpr int kKBlockBytes = kTileRows * 128;  // 128 rows x 64 bf16
-constexpr int kLag = 3;                        // pool gathers: stages of copies kept in flight
+constexpr int kLag = 4;                        // pool gathers: stages of copies kept in flight
 
 struct Params {
   const uint16_t* q;

@@ -258,6 +258,15 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, bool a_mn_ma
          | (static_cast<uint32_t>(M >> 4) << 24);    // M / 16
 }
 
+// Instruction descriptor, kind::f16: A = B = f16, D = f32, dense.
+__host__ __device__ constexpr uint32_t idesc_f16_f32(int M, int N, bool a_mn_major, bool b_mn_major) {
+  return (1u << 4)                                   // D format f32
+         | (static_cast<uint32_t>(a_mn_major) << 15) // A major (A, B format 0: f16)
+         | (static_cast<uint32_t>(b_mn_major) << 16) // B major
+         | (static_cast<uint32_t>(N >> 3) << 17)     // N / 8
+         | (static_cast<uint32_t>(M >> 4) << 24);    // M / 16
+}
+
 // Byte offset of the 16-byte chunk `chunk` (0..7) of row `row` inside a
 // 128-byte-swizzled region whose rows are 128 bytes apart.
 __host__ __device__ __forceinline__ uint32_t sw128_offset(uint32_t row, uint32_t chunk) {

@@ -750,8 +750,16 @@ csa2_status launch_variant(ClParams p, int64_t rows, cudaStream_t stream) {
 
 }  // namespace
 
+// Clusters of 8 CTAs win while they all run at once (a few rows; measured
+// on B200: 8 rows of 16384 keys in about 12 us, against 16 us on one CTA per
+// row).  With more rows they run in waves, and rows of at most
+// kSelectCtaMaxL keys go to one CTA each instead (32 rows of 16384: 35 ->
+// 18 us; 64 rows of 32768: 55 -> 22 us).
+constexpr int64_t kClusterMaxRows = 16;
+
 bool select_topk_cluster_applies(int64_t rows, int64_t L, int count0, int count1) {
   return count1 <= 0 && count0 > 0 && rows > 0 && rows < sm_count() && L > 0 &&
+         (rows <= kClusterMaxRows || L > kSelectCtaMaxL) &&
          L <= static_cast<int64_t>(kC) * kLargeChunk && !getenv("CSA2_TOPK_NO_CLUSTER");
 }
 
