@@ -212,13 +212,33 @@ __global__ void __launch_bounds__(kThreads, 1)
   // cover one 128-byte row segment
   const int et = (warp - 2) * 32 + lane;
   const int c16 = et & 7, grow0 = et >> 3;
-  // the first wave's row ids, loaded while the barriers and TMEM are set up
-  pdl_wait();                                  // the selection comes from the kernel before
-  int32_t first_ids[8];
-  if (warp >= 2 && n_waves > 0) {
+  // (grow0 + 16 i) & 7 == grow0 & 7: one swizzle per thread
+  const uint32_t swz = static_cast<uint32_t>((c16 ^ (grow0 & 7)) << 4);
+  auto issue_gather = [&](int64_t qi) {
+    const bool win_tile = tile >= p.T_sel;
+    const uint16_t* base = (win_tile ? p.win + (qi / p.Q) * p.win_rows * DV
+                                     : p.kv + (qi / p.Q) * p.n * DV) + c16 * 8;
+    int64_t off[8];
+    uint32_t nbytes[8];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) first_ids[i] = tile_row(p, slot, tile, grow0 + 16 * i);
-  }
+    for (int i = 0; i < 8; ++i) {
+      const int id = tile_row(p, qi, tile, grow0 + 16 * i);
+      off[i] = static_cast<int64_t>(id >= 0 ? id : 0) * DV;
+      nbytes[i] = id >= 0 ? 16u : 0u;            // empty slot: zero fill, nothing read
+    }
+#pragma unroll 1
+    for (int kb = 0; kb < kKB; ++kb) {          // not unrolled: one short body, re-executed
+#pragma unroll
+      for (int i = 0; i < 8; ++i)
+        cp_async_16(sKV + kb * kKBBytes + (grow0 + 16 * i) * 128 + swz, base + off[i] + kb * 64,
+                    nbytes[i]);
+      cp_async_commit();
+    }
+  };
+  // the first wave's rows are requested before the barriers and TMEM are set
+  // up (the copies need neither; they are published after the set-up)
+  pdl_wait();                                  // the selection comes from the kernel before
+  if (warp >= 2 && n_waves > 0) issue_gather(slot);
 
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
@@ -312,29 +332,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int row = quad * 32 + lane;                  // TMEM lane = tile row
     const uint32_t lane_off = static_cast<uint32_t>(quad * 32) << 16;
     const int hb = reduced_head_base(lane);
-    // (grow0 + 16 i) & 7 == grow0 & 7: one swizzle per thread
-    const uint32_t swz = static_cast<uint32_t>((c16 ^ (grow0 & 7)) << 4);
-    auto issue_gather = [&](int64_t qi, const int32_t* pre) {   // pre: this wave's ids, or null
-      const bool win_tile = tile >= p.T_sel;
-      const uint16_t* base = (win_tile ? p.win + (qi / p.Q) * p.win_rows * DV
-                                       : p.kv + (qi / p.Q) * p.n * DV) + c16 * 8;
-      int64_t off[8];
-      uint32_t nbytes[8];
-#pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        const int id = pre ? pre[i] : tile_row(p, qi, tile, grow0 + 16 * i);
-        off[i] = static_cast<int64_t>(id >= 0 ? id : 0) * DV;
-        nbytes[i] = id >= 0 ? 16u : 0u;            // empty slot: zero fill, nothing read
-      }
-#pragma unroll 1
-      for (int kb = 0; kb < kKB; ++kb) {          // not unrolled: one short body, re-executed
-#pragma unroll
-        for (int i = 0; i < 8; ++i)
-          cp_async_16(sKV + kb * kKBBytes + (grow0 + 16 * i) * 128 + swz, base + off[i] + kb * 64,
-                      nbytes[i]);
-        cp_async_commit();
-      }
-    };
     // each 64-column block is published once this thread's copies into it landed
     auto publish_gather = [&]() {
 #define CSA2_PUBLISH(KB)            \
@@ -345,10 +342,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       CSA2_PUBLISH(4) CSA2_PUBLISH(5) CSA2_PUBLISH(6) CSA2_PUBLISH(7)
 #undef CSA2_PUBLISH
     };
-    if (n_waves > 0) {
-      issue_gather(slot, first_ids);
-      publish_gather();
-    }
+    if (n_waves > 0) publish_gather();
     bool ok = true;
     for (int64_t w = 0; w < n_waves; ++w) {
       const int64_t qi = slot + w * p.G;
@@ -612,7 +606,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
         epi_bar();
-        if (more && ds + kStageDims >= d1) issue_gather(qi + p.G, nullptr);   // the KV region is free again
+        if (more && ds + kStageDims >= d1) issue_gather(qi + p.G);   // the KV region is free again
         // normalise, bf16, 8-byte stores of 4 dims
         const int pieces = nd / 4;
         for (int i = et; i < HA * pieces; i += 128) {
@@ -627,7 +621,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         epi_bar();
       }
-      if (more && d1 <= d0) issue_gather(qi + p.G, nullptr);
+      if (more && d1 <= d0) issue_gather(qi + p.G);
       if (tile == 0 && p.lse && et < HA)
         p.lse[qi * HA + et] = sML2[HA + et] > 0.0f ? sML2[et] + logf(sML2[HA + et]) : -INFINITY;
       // this CTA alone reads its dims of every partial: drop those lines from L2

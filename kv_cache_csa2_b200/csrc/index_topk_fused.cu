@@ -379,6 +379,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     int64_t it = 0;
     int cnt[NQ];
     uint32_t tau[NQ];
+    int64_t nvis[NQ];
     int64_t qrow0 = 0;                         // b * Q + g * NQ of the current group
     auto finish_group = [&]() {
       for (int qq = 0; qq < NQ; ++qq) {
@@ -416,6 +417,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int qq = 0; qq < NQ; ++qq) {
           cnt[qq] = 0;
           tau[qq] = 0u;
+          // entries [0, nvis) are visible to query qq of the group (none past
+          // the sequence's last query)
+          const bool real = (qrow0 % p.Q) + qq < p.Q;
+          nvis[qq] = !real ? 0 : p.n_visible ? std::min<int64_t>(p.n_visible[qrow0 + qq], p.N) : p.N;
         }
       }
       const int acc = static_cast<int>(it & 1);
@@ -423,30 +428,41 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_wait(&tfull[acc], (it >> 1) & 1, abort_flag, p.err);
       tc_fence_after();
       const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + acc * C::NCOL;
-      // (arrays over all NQ queries keep compile-time indices; this warp fills
-      // the QPW of its half, the branch being uniform over the warp)
+      // this warp's QPW queries, HP columns each, read in chunks of kChunk
+      // columns one chunk ahead of the arithmetic (a wait covers every load
+      // issued before it, so chunk c + 1 is requested after chunk c landed)
+      constexpr int kChunk = HP % 32 == 0 ? 32 : 16;
+      constexpr int kPerQ = HP / kChunk;
+      constexpr int kChunks = QPW * kPerQ;
+      const uint32_t tq = taddr + static_cast<uint32_t>(half * QPW * HP);
+      uint32_t v[2][kChunk];
+      auto load_chunk = [&](int c, uint32_t (&dst)[kChunk]) {
+        const uint32_t col = static_cast<uint32_t>((c / kPerQ) * HP + (c % kPerQ) * kChunk);
+        if constexpr (kChunk == 32) tmem_ld32(tq + col, dst);
+        else tmem_ld16(tq + col, dst);
+      };
+      float a[QPW];
+#pragma unroll
+      for (int j = 0; j < QPW; ++j) a[j] = 0.0f;
+      const float* wq = sW + half * QPW * HP;
+      load_chunk(0, v[0]);
+#pragma unroll
+      for (int c = 0; c < kChunks; ++c) {
+        tmem_wait_ld();
+        if (c + 1 < kChunks) load_chunk(c + 1, v[(c + 1) & 1]);
+        const int j = c / kPerQ, h0 = (c % kPerQ) * kChunk;
+#pragma unroll
+        for (int h = 0; h < kChunk; ++h) {
+          float x = __uint_as_float(v[c & 1][h]);
+          if (p.relu) x = fmaxf(x, 0.0f);
+          a[j] = fmaf(wq[j * HP + h0 + h], x, a[j]);
+        }
+      }
+      // (arrays over all NQ queries keep compile-time indices; the branch on
+      // the warp's half is uniform over the warp)
       float s[NQ];
 #pragma unroll
-      for (int qq = 0; qq < NQ; ++qq) {
-        s[qq] = 0.0f;
-        if (qq / QPW != half) continue;
-        float a = 0.0f;
-        constexpr int kChunk = HP % 32 == 0 ? 32 : 16;    // columns per TMEM load
-#pragma unroll
-        for (int h0 = 0; h0 < HP; h0 += kChunk) {
-          uint32_t v[kChunk];
-          if constexpr (kChunk == 32) tmem_ld32(taddr + qq * HP + h0, v);
-          else tmem_ld16(taddr + qq * HP + h0, v);
-          tmem_wait_ld();
-#pragma unroll
-          for (int h = 0; h < kChunk; ++h) {
-            float x = __uint_as_float(v[h]);
-            if (p.relu) x = fmaxf(x, 0.0f);
-            a = fmaf(sW[qq * HP + h0 + h], x, a);
-          }
-        }
-        s[qq] = a;
-      }
+      for (int qq = 0; qq < NQ; ++qq) s[qq] = qq / QPW == half ? a[qq % QPW] : 0.0f;
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&tempty[acc]);
@@ -459,10 +475,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         key[qq] = 0u;
         bal[qq] = 0u;
         if (qq / QPW != half) continue;
-        const int64_t qr = qrow0 + qq;
-        bool vis = e < p.N && (qrow0 % p.Q) + qq < p.Q;           // a query of this sequence
-        if (vis && p.n_visible) vis = e < p.n_visible[qr];
-        key[qq] = vis ? score_key(s[qq]) : 0u;
+        key[qq] = e < nvis[qq] ? score_key(s[qq]) : 0u;
         bal[qq] = __ballot_sync(0xffffffffu, key[qq] > tau[qq]);
         if (lane == 0) wc[quad * NQ + qq] = __popc(bal[qq]);
       }
