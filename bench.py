@@ -664,7 +664,7 @@ def run_reference(args, wl, world, rank):
 # ---------------------------------------------------------------------------- kernel cases
 
 KERNEL_CASES = ("attn", "full", "reindex", "attn_swa", "dense", "compress_hca", "full_fp4",
-                "reindex_fp4", "fused_prefill")
+                "reindex_fp4", "fused_prefill", "attn_prefill")
 
 
 def run_kernel_case(name, reps=4, timed=False):
@@ -682,7 +682,9 @@ def run_kernel_case(name, reps=4, timed=False):
       full_fp4       full with the FP4 indexer (FP4 q and K, bf16 scores)
       reindex_fp4    reindex with the FP4 indexer
       fused_prefill  csa2_index_topk(FULL) of a 4096-query prefill chunk over 262144
-                     entries, top 2048: the fused indexer + streaming top-k"""
+                     entries, top 2048: the fused indexer + streaming top-k
+      attn_prefill   csa2_sparse_attn of the same chunk: 4096 queries x 64 heads x 512,
+                     k = 2048 of 262144 entries each"""
     import torch
     import kv_cache_csa2_b200 as K
     g = torch.Generator(device="cuda").manual_seed(0)
@@ -709,6 +711,14 @@ def run_kernel_case(name, reps=4, timed=False):
             nbytes += B * 128 * D * 2
             flops += 4.0 * B * 128 * Ha * D
             call = lambda: K.csa2_sparse_attn_swa(q, kv, topk, D ** -0.5, win, we, 128)  # noqa: E731
+    elif name == "attn_prefill":
+        Q, N = 4096, 262144
+        kv, q = randn(1, N, D), randn(1, Q, Ha, D)
+        topk = torch.stack([torch.sort(torch.randperm(N, device="cuda", generator=g)[:k_sel])[0]
+                            for _ in range(Q)]).view(1, Q, k_sel).to(torch.int32)
+        nbytes = Q * k_sel * (D * 2 + 4) + Q * Ha * (D * 4 + 4)
+        flops = 4.0 * Q * k_sel * Ha * D
+        call = lambda: K.csa2_sparse_attn(q, kv, topk, D ** -0.5)  # noqa: E731
     elif name == "dense":
         N = 8192
         kv, q = randn(B, N, D), randn(B, 1, Ha, D)

@@ -40,19 +40,15 @@
 
 #include "common.cuh"
 #include "launchers.h"
+#include "attn_common.cuh"
 #include "sm100.cuh"
 
 namespace csa2 {
 namespace {
 using namespace sm100;
+using namespace attn;
 
-constexpr int HA = 64;
-constexpr int DV = 512;
-constexpr int kRows = 128;                    // rows per tile (MMA M of S^T)
 constexpr int kThreads = 6 * 32;
-constexpr int kKB = DV / 64;                  // 8 K-blocks of 64 dims
-constexpr int kKBBytes = kRows * 128;         // 16 KiB
-constexpr int kMaxTiles = 64;                 // k <= 8192
 constexpr int kPartFloats = DV * HA;          // partial O^T [dim][head], 128 KiB
 constexpr int kSlotFloats = kPartFloats + 2 * HA;   // + the tile's m[HA], l[HA]
 
@@ -97,76 +93,12 @@ struct Params {
   unsigned wait_offset;            // added to the awaited count (0, or unreachable for tests)
 };
 
-// Reduce 64 per-thread values over the 32 lanes of a warp (max or sum): five
-// exchange steps, each halving the values a lane keeps; on return v[0], v[1]
-// hold heads base, base+1 with base = reduced_head_base(lane).
-template <bool MAX>
-__device__ __forceinline__ void warp_transpose_reduce(float (&v)[64], int lane) {
-#pragma unroll
-  for (int step = 0; step < 5; ++step) {
-    const int half = 32 >> step;           // values kept after this step
-    const int ofs = 16 >> step;            // partner lane distance
-    const bool upper = lane & ofs;
-#pragma unroll
-    for (int i = 0; i < half; ++i) {
-      const float keep = upper ? v[i + half] : v[i];
-      const float give = upper ? v[i] : v[i + half];
-      const float got = __shfl_xor_sync(0xffffffffu, give, ofs);
-      v[i] = MAX ? fmaxf(keep, got) : keep + got;
-    }
-  }
-}
-// Max of one float over the 32 lanes of a warp (every lane gets it).
-__device__ __forceinline__ float warp_max_f32(float v) {
-  float r;
-  asm volatile("redux.sync.max.f32 %0, %1, 0xffffffff;" : "=f"(r) : "f"(v));
-  return r;
-}
-
-__device__ __forceinline__ int reduced_head_base(int lane) {
-  return ((lane >> 4) & 1) * 32 + ((lane >> 3) & 1) * 16 + ((lane >> 2) & 1) * 8 +
-         ((lane >> 1) & 1) * 4 + (lane & 1) * 2;
-}
-
 __device__ __forceinline__ void epi_bar() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
-
-// weight of a partial with max m in a sum whose max is M (0 for empty partials)
-__device__ __forceinline__ float rescale(float m, float M) {
-  return (m == -INFINITY || M == -INFINITY) ? 0.0f : __expf(m - M);
-}
 
 __device__ __forceinline__ unsigned ld_acquire_u32(const unsigned* p) {
   unsigned v;
   asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
   return v;
-}
-
-// Row of its source that row r of tile `tile` of query qi reads, or -1 for
-// an empty slot: a selected entry (tile < T_sel: the selection list, or the
-// slot itself when dense), or a window row (tile == T_sel).  An index
-// outside its source is recorded and treated as empty.
-__device__ __forceinline__ int tile_row(const Params& p, int64_t qi, int tile, int r) {
-  if (tile < p.T_sel) {
-    const int64_t pos = static_cast<int64_t>(tile) * kRows + r;
-    if (pos >= p.k) return -1;
-    if (!p.topk) {
-      const int64_t vis = p.n_vis ? p.n_vis[qi] : p.k;
-      return pos < vis ? static_cast<int>(pos) : -1;
-    }
-    const int id = p.topk[qi * p.k + pos];
-    if (id >= p.n || id < -1) {
-      raise_dev_error(p.err, DEVERR_BOUNDS);
-      return -1;
-    }
-    return id;
-  }
-  const int e = p.win_end[qi];
-  if (e < 0 || e > p.win_rows) {
-    raise_dev_error(p.err, DEVERR_BOUNDS);
-    return -1;
-  }
-  const int row = e - p.W + r;
-  return (r < p.W && row >= 0) ? row : -1;
 }
 
 // Drops a 128-byte line from L2 without writing it back (its content becomes
@@ -187,8 +119,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   float* sML = reinterpret_cast<float*>(smem + OFF_ML);      // m[HA], l[HA] of this tile
   float* sML2 = reinterpret_cast<float*>(smem + OFF_ML2);    // M[HA], L[HA] of the query
   float* sStage = reinterpret_cast<float*>(sQ);              // [HA][kStageStride]
-  float* sW = reinterpret_cast<float*>(sQ + kWeightsOff);    // [T][HA] weights
-  float* sLv = sW + kMaxTiles * HA;                          // [T][HA] row sums l_j
+  float* sW = reinterpret_cast<float*>(sQ + kWeightsOff);    // [T][HA] combine factors a_j
+  float* sLv = sW + kMaxTiles * HA;                          // [T][HA] combine factors b_j
   uint64_t* bar = reinterpret_cast<uint64_t*>(smem + OFF_BAR);
   uint64_t* q_full = bar + 0;
   uint64_t* s_full = bar + 1;
@@ -331,7 +263,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int ew = warp - 2;                           // epilogue warp 0..3
     const int row = quad * 32 + lane;                  // TMEM lane = tile row
     const uint32_t lane_off = static_cast<uint32_t>(quad * 32) << 16;
-    const int hb = reduced_head_base(lane);
+    const int hb = 2 * lane;                         // the heads lane reduces last
     // each 64-column block is published once this thread's copies into it landed
     auto publish_gather = [&]() {
 #define CSA2_PUBLISH(KB)            \
@@ -358,8 +290,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_wait_ld();
 #pragma unroll
         for (int h = 0; h < 32; ++h) {
-          x[h] = valid ? p.scale * __uint_as_float(v0[h]) : -INFINITY;
-          x[32 + h] = valid ? p.scale * __uint_as_float(v1[h]) : -INFINITY;
+          x[h] = scaled_score(valid, p.scale, v0[h]);
+          x[32 + h] = scaled_score(valid, p.scale, v1[h]);
         }
       } else {
 #pragma unroll
@@ -387,8 +319,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int u = 0; u < 2; ++u) {
             const int h = 4 * h4 + 2 * u;
-            const float e0 = (x[h] == -INFINITY) ? 0.0f : __expf(x[h] - mm[2 * u]);
-            const float e1 = (x[h + 1] == -INFINITY) ? 0.0f : __expf(x[h + 1] - mm[2 * u + 1]);
+            const float e0 = p_value(x[h], mm[2 * u]);
+            const float e1 = p_value(x[h + 1], mm[2 * u + 1]);
             const uint32_t pk = pack_bf16x2(e0, e1);
             packed[2 * h4 + u] = pk;
             lsum[h] = bf16_lo(pk);
@@ -403,11 +335,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(p_full);
-      warp_transpose_reduce<false>(lsum, lane);
+      warp_transpose_reduce<HA, false>(lsum, lane);
       sRed[ew * HA + hb] = lsum[0];
       sRed[ew * HA + hb + 1] = lsum[1];
       epi_bar();
-      if (et < HA) sML[HA + et] = (sRed[et] + sRed[HA + et]) + (sRed[2 * HA + et] + sRed[3 * HA + et]);
+      if (et < HA) sML[HA + et] = quad_sum(sRed[et], sRed[HA + et], sRed[2 * HA + et], sRed[3 * HA + et]);
       // partial (O^T, m, l) of this tile to workspace slot (buffer w & 1, CTA).
       // O^T is staged in the KV region as [dim][16 chunks of 4 heads] with
       // chunk h4 at position h4 ^ (dim & 7) (conflict-free) and written with
@@ -479,64 +411,36 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       epi_bar();
-      // weights of the T partials exp(m_j - M), the query's M and L
-      if (p.bulk) {
-        // the copies read memory that exists whatever the flags said, so they
-        // all land: wait for them also after a give-up (bounded: 0.1 s), so
-        // that no copy is in flight when the region is reused or the CTA exits
-        {
+      // the tile-order combine factors (a_j, b_j) of every head, the query's M and L
+      {
+        if (p.bulk) {
+          // the copies read memory that exists whatever the flags said, so they
+          // all land: wait for them also after a give-up (bounded: 0.1 s), so
+          // that no copy is in flight when the region is reused or the CTA exits
           const uint64_t t0 = globaltimer_ns();
           bool landed;
           while (!(landed = mbar_try_wait(r_full, par)) && globaltimer_ns() - t0 < 100000000ull) {
           }
           ok = ok && landed;
-        }
-        // all 128 threads: head h = et % 64 takes tiles j = half, half + 2, ...
-        // (half = et / 64); every load is issued before any is used
-        {
-          const int h = et & (HA - 1), half = et >> 6;
-          const uint32_t mlj = smem_u32(sP) + h * 4;    // m_j at + j*512, l_j at + j*512 + 256
-          float mj[16], lj[16];                          // T <= 32: at most 16 tiles per half
-#pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            const int j = half + 2 * i;
-            mj[i] = j < p.T ? lds_f32(mlj + j * 2 * HA * 4) : -INFINITY;
-            lj[i] = j < p.T ? lds_f32(mlj + j * 2 * HA * 4 + HA * 4) : 0.0f;
-          }
-          float mh = -INFINITY;
-#pragma unroll
-          for (int i = 0; i < 16; ++i) mh = fmaxf(mh, mj[i]);
-          sRed[half * HA + h] = mh;
-          epi_bar();
-          const float M = fmaxf(sRed[h], sRed[HA + h]);
-          float Lh = 0.0f;                               // this half's tiles, in tile order
-#pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            const float wj = rescale(mj[i], M);
-            if (half + 2 * i < p.T) sW[(half + 2 * i) * HA + h] = wj;
-            Lh += lj[i] * wj;
-          }
-          sRed[2 * HA + half * HA + h] = Lh;
-          epi_bar();
-          if (et < HA) {
-            sML2[et] = M;
-            sML2[HA + et] = sRed[2 * HA + et] + sRed[3 * HA + et];   // even tiles, then odd tiles
-          }
-        }
-      } else {
-        float* dstv = et < HA ? sW : sLv;                // m_j into sW, l_j into sLv
+        } else {
+          // (m_j, l_j) of every tile into sW (m) and sLv (l)
+          float* dstv = et < HA ? sW : sLv;
 #pragma unroll 8
-        for (int j = 0; j < p.T; ++j)
-          dstv[j * HA + (et & (HA - 1))] = __ldcg(pb + static_cast<int64_t>(j) * kSlotFloats + kPartFloats + et);
-        epi_bar();
+          for (int j = 0; j < p.T; ++j)
+            dstv[j * HA + (et & (HA - 1))] = __ldcg(pb + static_cast<int64_t>(j) * kSlotFloats + kPartFloats + et);
+          epi_bar();
+        }
         if (et < HA) {
-          float M = -INFINITY;
-          for (int j = 0; j < p.T; ++j) M = fmaxf(M, sW[j * HA + et]);
-          float L = 0.0f;
+          // m_j, l_j: on the bulk path in the P region (tile j at j * 512 bytes:
+          // m then l), else in sW / sLv; a_j over m_j in sW, b_j over l_j in sLv
+          const uint32_t mlb = smem_u32(sP) + et * 4;
+          float M = -INFINITY, L = 0.0f;
           for (int j = 0; j < p.T; ++j) {
-            const float wj = rescale(sW[j * HA + et], M);
-            sW[j * HA + et] = wj;
-            L += sLv[j * HA + et] * wj;
+            const float mj = p.bulk ? lds_f32(mlb + j * 2 * HA * 4) : sW[j * HA + et];
+            const float lj = p.bulk ? lds_f32(mlb + j * 2 * HA * 4 + HA * 4) : sLv[j * HA + et];
+            const float2 ab = combine_step(M, L, mj, lj);
+            sW[j * HA + et] = ab.x;
+            sLv[j * HA + et] = ab.y;
           }
           sML2[et] = M;
           sML2[HA + et] = L;
@@ -544,7 +448,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       epi_bar();
       // this CTA's output dims: sum over the partials in tile order
-      const uint32_t w0 = smem_u32(sW);
+      const uint32_t w0 = smem_u32(sW), l0 = smem_u32(sLv);
       for (int ds = d0; ds < d1; ds += kStageDims) {
         const int nd = min(kStageDims, d1 - ds);
         const int nch = nd * (HA / 4);                 // float4 chunks (dim, 4 heads)
@@ -568,13 +472,14 @@ __global__ void __launch_bounds__(kThreads, 1)
               float4 v[4];
 #pragma unroll
               for (int u = 0; u < 4; ++u) v[u] = lds_v4f(kv0 + j * slice_bytes + (in[u] ? off[u] : 0));
-              const float4 wj = lds_v4f(w0 + (j * HA + 4 * h4) * 4);
+              const float4 aj = lds_v4f(w0 + (j * HA + 4 * h4) * 4);
+              const float4 bj = lds_v4f(l0 + (j * HA + 4 * h4) * 4);
 #pragma unroll
               for (int u = 0; u < 4; ++u) {
-                acc[u].x += v[u].x * wj.x;
-                acc[u].y += v[u].y * wj.y;
-                acc[u].z += v[u].z * wj.z;
-                acc[u].w += v[u].w * wj.w;
+                acc[u].x = combine_acc(acc[u].x, v[u].x, aj.x, bj.x);
+                acc[u].y = combine_acc(acc[u].y, v[u].y, aj.y, bj.y);
+                acc[u].z = combine_acc(acc[u].z, v[u].z, aj.z, bj.z);
+                acc[u].w = combine_acc(acc[u].w, v[u].w, aj.w, bj.w);
               }
             }
           } else {
@@ -584,13 +489,14 @@ __global__ void __launch_bounds__(kThreads, 1)
               float4 v[4];
 #pragma unroll
               for (int u = 0; u < 4; ++u) v[u] = __ldcg(reinterpret_cast<const float4*>(sj + (in[u] ? off[u] : 0)));
-              const float4 wj = *reinterpret_cast<const float4*>(sW + j * HA + 4 * h4);
+              const float4 aj = *reinterpret_cast<const float4*>(sW + j * HA + 4 * h4);
+              const float4 bj = *reinterpret_cast<const float4*>(sLv + j * HA + 4 * h4);
 #pragma unroll
               for (int u = 0; u < 4; ++u) {
-                acc[u].x += v[u].x * wj.x;
-                acc[u].y += v[u].y * wj.y;
-                acc[u].z += v[u].z * wj.z;
-                acc[u].w += v[u].w * wj.w;
+                acc[u].x = combine_acc(acc[u].x, v[u].x, aj.x, bj.x);
+                acc[u].y = combine_acc(acc[u].y, v[u].y, aj.y, bj.y);
+                acc[u].z = combine_acc(acc[u].z, v[u].z, aj.z, bj.z);
+                acc[u].w = combine_acc(acc[u].w, v[u].w, aj.w, bj.w);
               }
             }
           }
@@ -611,19 +517,18 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int pieces = nd / 4;
         for (int i = et; i < HA * pieces; i += 128) {
           const int h = i / pieces, pc = i % pieces;
-          const float L = sML2[HA + h];
-          const float inv = L > 0.0f ? 1.0f / L : 0.0f;
+          const float inv = inv_sum(sML2[HA + h]);
           const float* a = sStage + h * kStageStride + 4 * pc;
           uint2 o;
-          o.x = pack_bf16x2(a[0] * inv, a[1] * inv);
-          o.y = pack_bf16x2(a[2] * inv, a[3] * inv);
+          o.x = pack_bf16x2(__fmul_rn(a[0], inv), __fmul_rn(a[1], inv));
+          o.y = pack_bf16x2(__fmul_rn(a[2], inv), __fmul_rn(a[3], inv));
           *reinterpret_cast<uint2*>(p.out + (qi * HA + h) * DV + ds + 4 * pc) = o;
         }
         epi_bar();
       }
       if (more && d1 <= d0) issue_gather(qi + p.G);
       if (tile == 0 && p.lse && et < HA)
-        p.lse[qi * HA + et] = sML2[HA + et] > 0.0f ? sML2[et] + logf(sML2[HA + et]) : -INFINITY;
+        p.lse[qi * HA + et] = lse_of(sML2[et], sML2[HA + et]);
       // this CTA alone reads its dims of every partial: drop those lines from L2
       if (d1 > d0) {
         const int lines = static_cast<int>(slice_bytes / 128);
@@ -719,6 +624,8 @@ csa2_status launch_sparse_attn_tc(const void* q, const csa2_kv& kv, const int32_
   if (!applies(Ha, kv.dim, k, kv.fmt, win)) return CSA2_ERR_UNSUPPORTED;
   const int64_t n_queries = static_cast<int64_t>(B) * Q;
   if (n_queries * HA > 0x7fffffffLL) return CSA2_ERR_UNSUPPORTED;
+  if (sparse_attn_seq_applies(n_queries, k, win))       // many queries: one CTA per query
+    return launch_sparse_attn_seq(q, kv, topk, B, Q, k, scale, out, lse, stream, rows);
   const Shape s = shape_for(k, win);
   const int cap = resident_ctas();
   if (cap < s.T) return CSA2_ERR_UNSUPPORTED;

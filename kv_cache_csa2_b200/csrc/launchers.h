@@ -111,6 +111,15 @@ struct AttnRows {
 };
 constexpr int kMaxWindow = 128;
 
+// The tensor-core attention for 64 heads x 512 in two schedules with the same
+// arithmetic per query (bit for bit): a query's tiles on several CTAs
+// (attn_tc.cu, few queries) or in sequence on one CTA (attn_seq.cu, many
+// queries; no workspace).  CSA2_ATTN_SEQ=0 / 1 forces the choice.
+bool sparse_attn_seq_applies(int64_t n_queries, int k, bool win);
+csa2_status launch_sparse_attn_seq(const void* q, const csa2_kv& kv, const int32_t* topk, int B,
+                                   int Q, int k, float scale, void* out, float* lse,
+                                   cudaStream_t stream, const AttnRows& rows);
+
 size_t sparse_attn_workspace(int B, int Q, int Ha, int D, int k, csa2_kv_fmt fmt, bool window = false);
 // sync_zeroed: kAttnMaxGrid * 8 bytes of per-CTA flags that were zero before
 // their first use and are left consistent by every launch (a layer group's),
