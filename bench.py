@@ -175,10 +175,16 @@ PROFILED_SOURCES = {
 }
 
 
-def ncu_traffic(kind):
+# the workload the committed summaries were captured on (traffic per launch
+# depends on the workload's sizes)
+PROFILED_WORKLOAD = "c4_hier_decode_f_3ri_4u_1m"
+
+
+def ncu_traffic(kind, workload):
     """DRAM bytes per launch for `kind` from the committed ncu summary, or None
-    when there is none or the kernel source changed since it was taken."""
-    if kind not in PROFILED_SOURCES:
+    when there is none, it was taken on another workload, or the kernel
+    source changed since it was taken."""
+    if kind not in PROFILED_SOURCES or workload != PROFILED_WORKLOAD:
         return None
     srcs, path = PROFILED_SOURCES[kind]
     try:
@@ -504,13 +510,13 @@ def run_ours(args, wl, world, rank, local):
         if tensor:
             achieved = flops_per_launch / avg_s / 1e12 if avg_s > 0 else 0.0
             roof = {"kernel": dom, "bound": "tensor", "achieved": round(achieved, 1), "peak": tflops,
-                    "unit": "TFLOP/s", "frac": round(achieved / tflops, 4), "traffic": ncu_traffic(dom),
+                    "unit": "TFLOP/s", "frac": round(achieved / tflops, 4), "traffic": ncu_traffic(dom, wl.name),
                     "algorithmic_flops_per_launch": int(flops_per_launch),
                     "algorithmic_bytes_per_launch": int(bytes_per_launch), "peak_source": tf_src}
         else:
             achieved = bytes_per_launch / avg_s / 1e9 if avg_s > 0 else 0.0
             roof = {"kernel": dom, "bound": "hbm", "achieved": round(achieved, 1), "peak": hbm,
-                    "unit": "GB/s", "frac": round(achieved / hbm, 4), "traffic": ncu_traffic(dom),
+                    "unit": "GB/s", "frac": round(achieved / hbm, 4), "traffic": ncu_traffic(dom, wl.name),
                     "algorithmic_bytes_per_launch": int(bytes_per_launch),
                     "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs)" if peak_src == "measured"
                     else "fallback 6650 GB/s"}
