@@ -670,7 +670,7 @@ def run_reference(args, wl, world, rank):
 # ---------------------------------------------------------------------------- kernel cases
 
 KERNEL_CASES = ("attn", "full", "reindex", "attn_swa", "dense", "compress_hca", "full_fp4",
-                "reindex_fp4", "fused_prefill", "attn_prefill")
+                "reindex_fp4", "fused_prefill", "fused_small", "attn_prefill")
 
 
 def run_kernel_case(name, reps=4, timed=False):
@@ -689,6 +689,8 @@ def run_kernel_case(name, reps=4, timed=False):
       reindex_fp4    reindex with the FP4 indexer
       fused_prefill  csa2_index_topk(FULL) of a 4096-query prefill chunk over 262144
                      entries, top 2048: the fused indexer + streaming top-k
+      fused_small    the fused indexer on 592 queries (one 4-query group per SM) over 65536
+                     entries, top 2048 (the size its ncu capture uses)
       attn_prefill   csa2_sparse_attn of the same chunk: 4096 queries x 64 heads x 512,
                      k = 2048 of 262144 entries each"""
     import torch
@@ -738,6 +740,14 @@ def run_kernel_case(name, reps=4, timed=False):
         bias = torch.randn(m, D, device="cuda", generator=g)
         nbytes = B * T * D * 6 + B * (T // m) * D * 2 + m * D * 4
         call = lambda: K.csa2_compress_hca(c, z, bias, m)  # noqa: E731
+    elif name == "fused_small":
+        Q, N = 592, 65536
+        q = randn(1, Q, 64, 128)
+        w = torch.randn(1, Q, 64, device="cuda", generator=g)
+        kk = randn(1, N, 128)
+        flops = 2.0 * 64 * 128 * Q * N
+        nbytes = N * 128 * 2 + Q * 64 * (128 * 2 + 4) + Q * k_sel * 4
+        call = lambda: K.csa2_index_topk(K.FULL, q, w, kk, k_sel)  # noqa: E731
     elif name == "fused_prefill":
         Q, N = 4096, 262144
         q = randn(1, Q, 64, 128)
