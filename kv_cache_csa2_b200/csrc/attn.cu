@@ -10,6 +10,8 @@
 // It serves every shape; the tensor-core kernel in attn_tc.cu takes the
 // shapes it supports.  The reduction order per query is fixed (rows in list
 // order, 16 at a time), so a query's result does not depend on B or Q.
+#include <algorithm>
+
 #include "common.cuh"
 #include "launchers.h"
 
@@ -371,7 +373,10 @@ csa2_status run_simt(const void* q, const csa2_kv& kv, const int32_t* topk, int 
 size_t sparse_attn_workspace(int B, int Q, int Ha, int D, int k, csa2_kv_fmt fmt, bool window) {
   const size_t tc = sparse_attn_tc_workspace(B, Q, Ha, D, k, fmt, window);
   if (tc > 0) return tc;
-  return split_for(static_cast<int64_t>(B) * Q, Ha, D, k, window, kMaxWindow).bytes;
+  const size_t simt = split_for(static_cast<int64_t>(B) * Q, Ha, D, k, window, kMaxWindow).bytes;
+  if (sparse_attn_narrow_applies(Ha, D, k, window))
+    return std::max(simt, sparse_attn_narrow_workspace(B, Q, Ha, k, window));
+  return simt;
 }
 
 csa2_status launch_sparse_attn(const void* q, const csa2_kv& kv, const int32_t* topk, int B,
@@ -383,6 +388,11 @@ csa2_status launch_sparse_attn(const void* q, const csa2_kv& kv, const int32_t* 
                                         sync_zeroed, stream, rows);
   if (s != CSA2_ERR_UNSUPPORTED) return s;
   const int D = kv.dim;
+  if (sparse_attn_narrow_applies(Ha, D, k, rows.win != nullptr)) {
+    s = launch_sparse_attn_narrow(q, kv, topk, B, Q, Ha, k, scale, out, lse, ws, ws_bytes, sync_zeroed,
+                                  stream, rows);
+    if (s != CSA2_ERR_UNSUPPORTED) return s;
+  }
 #define CSA2_SIMT(HA_, D_)                                                                       \
   if (Ha == HA_ && D == D_)                                                                      \
     return run_simt<HA_, D_>(q, kv, topk, B, Q, k, scale, out, lse, ws, ws_bytes, sync_zeroed, stream, rows);

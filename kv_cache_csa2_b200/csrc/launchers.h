@@ -115,6 +115,14 @@ constexpr int kMaxWindow = 128;
 // arithmetic per query (bit for bit): a query's tiles on several CTAs
 // (attn_tc.cu, few queries) or in sequence on one CTA (attn_seq.cu, many
 // queries; no workspace).  CSA2_ATTN_SEQ=0 / 1 forces the choice.
+// Entries of width 128 (16, 32 or 64 heads, bf16 or FP4 rows) on the tensor
+// cores (attn_narrow.cu); CSA2_ATTN_SIMT forces the CUDA-core kernel.
+bool sparse_attn_narrow_applies(int Ha, int D, int k, bool win);
+size_t sparse_attn_narrow_workspace(int B, int Q, int Ha, int k, bool win);
+csa2_status launch_sparse_attn_narrow(const void* q, const csa2_kv& kv, const int32_t* topk, int B,
+                                      int Q, int Ha, int k, float scale, void* out, float* lse,
+                                      void* ws, size_t ws_bytes, unsigned long long* sync_zeroed,
+                                      cudaStream_t stream, const AttnRows& rows);
 bool sparse_attn_seq_applies(int64_t n_queries, int k, bool win);
 csa2_status launch_sparse_attn_seq(const void* q, const csa2_kv& kv, const int32_t* topk, int B,
                                    int Q, int k, float scale, void* out, float* lse,
