@@ -132,6 +132,35 @@ __global__ void __launch_bounds__(kThreads) attn_narrow_kernel(const Params p) {
   constexpr uint32_t S_COL = 0, O_COL = 64;             // S^T and O^T: HA columns each
 
   pdl_wait();                                           // the selection comes from the kernel before
+  // q and the tile's rows are requested before the barriers and TMEM are set
+  // up (warps 2-5; thread et takes row et); they land in shared memory after
+  const int et = (warp - 2) * 32 + lane;                // 0..127 in warps 2-5
+  const bool win_tile = tile >= p.T_sel;
+  constexpr int QPT = HA * 16 / 128;                    // 16-byte chunks of q per thread
+  uint4 qv[QPT];
+  uint4 codes[4] = {};
+  uint2 scl = make_uint2(0, 0);
+  int id = -1;
+  if (warp >= 2) {
+    const uint4* qg = reinterpret_cast<const uint4*>(p.q + qi * HA * DN);
+#pragma unroll
+    for (int j = 0; j < QPT; ++j) qv[j] = __ldg(qg + et + 128 * j);
+    id = tile_row(p, qi, tile, et);
+    if (!FP4 || win_tile) {
+      const uint16_t* src = win_tile ? p.win + (seq * p.win_rows + (id >= 0 ? id : 0)) * DN
+                                     : static_cast<const uint16_t*>(p.kv) + (seq * p.n + (id >= 0 ? id : 0)) * DN;
+#pragma unroll
+      for (int c = 0; c < 16; ++c)
+        cp_async_16(sKV + (c >> 3) * kKBBytes + swz(et, c & 7), src + c * 8, id >= 0 ? 16u : 0u);
+      cp_async_commit();
+    } else if (id >= 0) {
+      const int64_t r = seq * p.n + id;
+      const uint4* cg = reinterpret_cast<const uint4*>(static_cast<const uint8_t*>(p.kv) + r * (DN / 2));
+#pragma unroll
+      for (int j = 0; j < 4; ++j) codes[j] = __ldg(cg + j);
+      scl = __ldg(reinterpret_cast<const uint2*>(p.kv_scales + r * (DN / 16)));
+    }
+  }
   if (threadIdx.x == 0) {
     mbar_init(kv_full, 128);
     mbar_init(s_full, 1);
@@ -183,38 +212,17 @@ __global__ void __launch_bounds__(kThreads) attn_narrow_kernel(const Params p) {
     // ------------------------------------------------------------ gather, softmax, output
     const int quad = warp & 3;
     const int ew = warp - 2;                            // 0..3
-    const int et = ew * 32 + lane;                      // 0..127
     const int row = quad * 32 + lane;                   // TMEM lane = tile row (and O^T dim)
     const uint32_t lane_off = static_cast<uint32_t>(quad * 32) << 16;
-    // q: [HA heads][128 dims] in two 64-dim blocks, 16-byte chunks
-    {
-      const uint4* qg = reinterpret_cast<const uint4*>(p.q + qi * HA * DN);
-      for (int i = et; i < HA * 16; i += 128) {
-        const int h = i >> 4, c = i & 15;
-        *reinterpret_cast<uint4*>(sQ + (c >> 3) * L::QKB + swz(h, c & 7)) = __ldg(qg + i);
-      }
-    }
-    // rows: thread et takes row et of the tile
-    const bool win_tile = tile >= p.T_sel;
-    const int id = tile_row(p, qi, tile, et);
-    if (!FP4 || win_tile) {
-      const uint16_t* src = win_tile ? p.win + (seq * p.win_rows + (id >= 0 ? id : 0)) * DN
-                                     : static_cast<const uint16_t*>(p.kv) + (seq * p.n + (id >= 0 ? id : 0)) * DN;
+    // q: [HA heads][128 dims] in two 64-dim blocks of 16-byte chunks
 #pragma unroll
-      for (int c = 0; c < 16; ++c)
-        cp_async_16(sKV + (c >> 3) * kKBBytes + swz(et, c & 7), src + c * 8, id >= 0 ? 16u : 0u);
-      cp_async_commit();
+    for (int j = 0; j < QPT; ++j) {
+      const int i = et + 128 * j, h = i >> 4, c = i & 15;
+      *reinterpret_cast<uint4*>(sQ + (c >> 3) * L::QKB + swz(h, c & 7)) = qv[j];
+    }
+    if (!FP4 || win_tile) {
       cp_async_wait<0>();
     } else {
-      uint4 codes[4] = {};
-      uint2 scl = make_uint2(0, 0);
-      if (id >= 0) {
-        const int64_t r = seq * p.n + id;
-        const uint4* cg = reinterpret_cast<const uint4*>(static_cast<const uint8_t*>(p.kv) + r * (DN / 2));
-#pragma unroll
-        for (int j = 0; j < 4; ++j) codes[j] = __ldg(cg + j);
-        scl = __ldg(reinterpret_cast<const uint2*>(p.kv_scales + r * (DN / 16)));
-      }
       // chunk c holds channels 8c .. 8c+7: 4 code bytes of block c / 2
 #pragma unroll
       for (int c = 0; c < 16; ++c) {
