@@ -7,9 +7,12 @@
 // This file holds the CUDA-core kernel: one CTA per query, the query's heads
 // in shared memory, the selected rows staged 16 at a time (f32, padded
 // stride), an online softmax per head and the per-head outputs in registers.
-// It serves every shape; the tensor-core kernel in attn_tc.cu takes the
-// shapes it supports.  The reduction order per query is fixed (rows in list
-// order, 16 at a time), so a query's result does not depend on B or Q.
+// It serves every shape; the tensor-core kernels take the shapes they
+// support first (attn_tc.cu / attn_seq.cu: 64 heads x 512 bf16;
+// attn_narrow.cu: entries of width 128), so this kernel runs the rest (width
+// 512 with 16 or 32 heads, FP4 at 64 x 512).  The reduction order per query
+// is fixed (rows in list order, 16 at a time), so a query's result does not
+// depend on B or Q.
 #include <algorithm>
 
 #include "common.cuh"
