@@ -169,7 +169,7 @@ def source_digest(*names) -> str:
 # kernel kind -> (source files whose digest must match the profile, profile summary)
 PROFILED_SOURCES = {
     "index_scores": (("index_scores.cu", "index_scores_tc.cu"), "profiles/index_scores_c4.md"),
-    "attn": (("attn.cu", "attn_tc.cu", "attn_common.cuh"), "profiles/attn_c4.md"),
+    "attn": (("attn_tc.cu", "attn_common.cuh", "sm100.cuh", "common.cuh"), "profiles/attn_c4.md"),
     "topk": (("topk.cu", "topk_multi.cu", "topk_cta.cu", "topk_cluster.cu"), "profiles/topk_c4.md"),
     "index_pool": (("index_scores.cu", "index_scores_tc.cu"), "profiles/index_pool_c4.md"),
 }
