@@ -96,3 +96,18 @@ def test_workspace_queries():
     assert ws >= 8 * 262144 * 4
     assert lib.csa2_index_topk_workspace(8, 1, 262144, 16384, 2048, 0) >= 8 * 16384 * 4
     assert lib.csa2_select_topk_workspace(8, 262144, 2048) >= 0
+
+
+def test_attention_workspace_covers_every_schedule():
+    """The attention workspace query is the maximum over the kernels a call may
+    take: entries of width 128 with several 128-row tiles keep per-tile
+    partials (a 128 x heads f32 block plus m and l per head) and a counter
+    per query; one tile needs none."""
+    lib = K.lib()
+    fp4, bf16 = 1, 0
+    # 64 queries, 16 heads, k = 256: two tiles per query
+    need = 64 * 2 * (128 * 16 + 2 * 16) * 4 + 64 * 4
+    assert lib.csa2_sparse_attn_workspace(64, 1, 16, 128, 256, fp4) >= need
+    assert lib.csa2_sparse_attn_workspace(64, 1, 16, 128, 256, bf16) >= need
+    # 64 heads x 512 (the split schedule): a 128 KiB partial per CTA and a flag
+    assert lib.csa2_sparse_attn_workspace(8, 1, 64, 512, 2048, bf16) >= 16 * 128 * 1024
