@@ -118,6 +118,8 @@ def gpu_group(wl, inp):
             kw = dict(n_visible=nv)
         if mode != "reuse":
             kw.update(q_index=dev_bf16(L["q_index"]), w_index=dev(L["w_index"]))
+        if "win" in L:                         # the layer's sliding-window rows
+            kw["swa"] = (dev_bf16(L["win"]), dev(L["win_end"]), wl.swa)
         g.layer(i, dev_bf16(L["q_attn"]), out, lse, **kw)
         topk, pool = g.copy_selection()
         r = {"mode": mode, "topk": topk.cpu().numpy(), "out": host_bf16(out),
@@ -157,6 +159,8 @@ def oracle_group(wl, inp, sample=None):
         if "q_index" in L:
             d["q_index"] = O.bf16_bits_to_float(L["q_index"][:, sl])
             d["w_index"] = L["w_index"][:, sl].astype(np.float64)
+        if "win" in L:
+            d["swa"] = (O.bf16_bits_to_float(L["win"]), L["win_end"][:, sl], wl.swa)
         layers.append(d)
     nv = inp["n_visible"][:, sl] if inp["n_visible"] is not None else None
     ik = I.bf16_bits_to_f32(inp["index_k"])
@@ -164,17 +168,22 @@ def oracle_group(wl, inp, sample=None):
                        n_visible=nv), new
 
 
-def attn_on_selection(wl, kv, q_attn_bits, topk):
+def attn_on_selection(wl, kv, q_attn_bits, topk, win=None):
     """The attention kernel, through the C ABI, on a given selection (the
     oracle's) for the layer's queries: kv is the group's bf16 KV on the
     device (packed to FP4 here when the workload stores FP4), q_attn_bits the
-    queries [B, Qs, Ha, D] as bf16 bits, topk int [B, Qs, k]."""
+    queries [B, Qs, Ha, D] as bf16 bits, topk int [B, Qs, k]; win = (window
+    rows as bf16 bits, win_end) for a layer with the sliding-window branch."""
     kv_arg, scales = kv, None
     if wl.kv_fp4:
         kv_arg, scales = K.csa2_fp4_pack(kv)
-    out, lse = K.csa2_sparse_attn(dev_bf16(q_attn_bits), kv_arg,
-                                  dev(np.ascontiguousarray(topk, dtype=np.int32)), wl.attn_scale,
-                                  kv_scales=scales)
+    sel = dev(np.ascontiguousarray(topk, dtype=np.int32))
+    if win is not None:
+        out, lse = K.csa2_sparse_attn_swa(dev_bf16(q_attn_bits), kv_arg, sel, wl.attn_scale,
+                                          win=dev_bf16(win[0]), win_end=dev(np.ascontiguousarray(win[1])),
+                                          W=wl.swa, kv_scales=scales)
+    else:
+        out, lse = K.csa2_sparse_attn(dev_bf16(q_attn_bits), kv_arg, sel, wl.attn_scale, kv_scales=scales)
     return host_bf16(out), lse.cpu().numpy().astype(np.float64)
 
 
@@ -235,7 +244,9 @@ def compare_groups(wl, inp, gres, ores, sample=None, min_exact=0.5, kv=None):
         oi = o["o"][same]
         check_attn(gi, g["lse"][:, sl][same], oi, o["lse"][same], f"layer {i} ({mode})")
         if kv is not None:
-            q_bits = inp["layers"][i]["q_attn"][:, sl]
-            out_r, lse_r = attn_on_selection(wl, kv, q_bits, o["topk"])
+            L = inp["layers"][i]
+            q_bits = L["q_attn"][:, sl]
+            win = (L["win"], L["win_end"][:, sl]) if "win" in L else None
+            out_r, lse_r = attn_on_selection(wl, kv, q_bits, o["topk"], win=win)
             check_attn(out_r, lse_r, o["o"], o["lse"], f"layer {i} ({mode}) on the oracle's selection")
     return same

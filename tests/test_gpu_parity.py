@@ -374,7 +374,7 @@ def test_group_small(wl):
 
 
 @pytest.mark.slow
-@pytest.mark.parametrize("wl", [C.C1, C.C2, C.C3, C.C4], ids=["c1", "c2", "c3", "c4"])
+@pytest.mark.parametrize("wl", [C.C1, C.C2, C.C3, C.C4, C.C6], ids=["c1", "c2", "c3", "c4", "c6"])
 def test_group_full_size(wl):
     inp = I.make_inputs(wl)
     gres, kv = U.gpu_group(wl, inp)
